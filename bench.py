@@ -1,0 +1,548 @@
+#!/usr/bin/env python
+"""Benchmark of the Kascade hot path on B200.
+
+One step = one decode step of the 32-layer batch-16 / 32K-context workload
+(anchors [0, 2, 8, 13, 14], k = 3277, 27 reuse layers through head maps)
+followed by one 16K-token causal prefill through 4 layers (1 anchor,
+3 reuse).  Every anchor / Top-k / reuse call runs through libkascade.so.
+
+Prints ONE JSON line (rank 0).  `value` is decode attention microseconds per
+layer for the whole job (max-over-ranks step time / (32 layers x N ranks),
+N independent replicas); prefill ms/layer, HBM GB/s and the per-kernel split
+are extra keys.  Inputs (68.7 GB of KV cache) are far larger than L2.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kascade|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "decode attn µs/layer & HBM GB/s at 32K ctx; prefill attn ms/layer at 16K (1×B200)"
+UNIT = "us/layer"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="kascade", choices=["kascade", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--only", default="all", choices=["all", "decode", "prefill"])
+    ap.add_argument("--decode-layers", type=int, default=None,
+                    help="profiling aid: materialise fewer decode layers (not a bench number)")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            torch.cuda.set_device(self.local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                    device_id=torch.device("cuda", self.local))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, x: float) -> float:
+        if not self.pg:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+class Clocks:
+    """nvidia-smi sampling during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def start(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if not self.p:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.p.terminate()
+        self.p.wait()
+        self.f.flush()
+        rows = [r.split(",") for r in open(self.f.name).read().strip().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------------------
+def build_decode(dev, n_layers=None):
+    from long_context_emitting_b200 import workload
+    from long_context_emitting_b200.schedule import DecodeSchedule
+
+    cfg = workload.DECODE_32K
+    L = cfg.n_layers if n_layers is None else n_layers
+    lens = cfg.seq_lens()
+    sch = DecodeSchedule(cfg.B, cfg.Hq, cfg.Hkv, lens, cfg.anchors, L, dev)
+    layers = [workload.decode_layer(cfg, l, dev) for l in range(L)]
+    maps = {l: workload.head_map(cfg, l).to(dev) for l in range(L) if l not in cfg.anchors}
+    outs = [torch.empty(cfg.B, cfg.Hq, cfg.d, dtype=torch.bfloat16, device=dev) for _ in range(L)]
+    return cfg, sch, layers, maps, outs
+
+
+def build_prefill(dev):
+    from long_context_emitting_b200 import workload
+    from long_context_emitting_b200.schedule import PrefillSchedule
+
+    cfg = workload.PREFILL_16K
+    sch = PrefillSchedule(cfg.B, cfg.Hq, cfg.Hkv, cfg.N, cfg.anchors, cfg.n_layers, dev)
+    layers = [workload.prefill_layer(cfg, l, dev) for l in range(cfg.n_layers)]
+    maps = {l: workload.head_map(cfg, l).to(dev) for l in range(cfg.n_layers) if l not in cfg.anchors}
+    outs = [torch.empty_like(layers[l]["q"]) for l in range(cfg.n_layers)]
+    return cfg, sch, layers, maps, outs
+
+
+class OpTimer:
+    """CUDA events around each call on the launching (current) stream."""
+
+    def __init__(self):
+        self.pending = []
+        self.times = {}
+
+    def run(self, name, fn, *args):
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record()
+        fn(*args)
+        e.record()
+        self.pending.append((name, s, e))
+
+    def collect(self):
+        torch.cuda.synchronize()
+        for name, s, e in self.pending:
+            self.times.setdefault(name, []).append(s.elapsed_time(e))
+        self.pending.clear()
+
+    def mean_ms(self, name):
+        v = self.times.get(name, [])
+        return sum(v) / len(v) if v else 0.0
+
+    def total_ms(self, name):
+        return sum(self.times.get(name, []))
+
+
+def decode_step(sch, layers, maps, outs, timer=None):
+    for l in range(sch.n_layers):
+        if sch.is_anchor(l):
+            if timer:
+                timer.run("dec_anchor", sch.run_anchor, layers[l], outs[l])
+                timer.run("dec_topk", sch.run_topk)
+            else:
+                sch.run_anchor(layers[l], outs[l])
+                sch.run_topk()
+        else:
+            if timer:
+                timer.run("dec_reuse", sch.run_reuse, layers[l], maps[l], outs[l])
+            else:
+                sch.run_reuse(layers[l], maps[l], outs[l])
+
+
+def prefill_step(sch, layers, maps, outs, timer=None):
+    for l in range(sch.n_layers):
+        if sch.is_anchor(l):
+            if timer:
+                timer.run("pre_anchor", sch.run_anchor, layers[l], outs[l])
+                timer.run("pre_topk", sch.run_topk)
+            else:
+                sch.run_anchor(layers[l], outs[l])
+                sch.run_topk()
+        else:
+            if timer:
+                timer.run("pre_reuse", sch.run_reuse, layers[l], maps[l], outs[l])
+            else:
+                sch.run_reuse(layers[l], maps[l], outs[l])
+
+
+# --------------------------------------------------------------------------------------
+def cpu_sample(steps: int = 1):
+    """The float64 oracle on a bounded sample of the same workload (host cores).
+
+    Decode: one anchor layer (attention + pooled + Top-k) and one reuse layer
+    for one sequence of the batch-16 / 32K workload, scaled to the batch and
+    the 5-anchor / 27-reuse mix.  Prefill: 2 query tiles x 1 KV head of the
+    16K anchor and reuse layers, scaled by causal key-pair counts.
+    Returns (decode us/layer, prefill ms/layer, sample description, cores)."""
+    import oracle as O
+    from long_context_emitting_b200 import workload
+
+    cores = len(os.sched_getaffinity(0))
+    torch.set_num_threads(cores)
+    cfg = workload.DECODE_32K
+    scale = 1.0 / np.sqrt(cfg.d)
+    a_in = workload.decode_sequence(cfg, 0, 0)
+    r_in = workload.decode_sequence(cfg, 1, 0)
+    q = a_in["q"].float().numpy()[None]
+    k = [a_in["k"].float().numpy()]
+    v = [a_in["v"].float().numpy()]
+    qr = r_in["q"].float().numpy()[None]
+    kr = [r_in["k"].float().numpy()]
+    vr = [r_in["v"].float().numpy()]
+    T = a_in["T"]
+    kk = O.k_for_len(T)
+    hm = workload.head_map(cfg, 1).numpy()
+    t_a = t_r = 0.0
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        _, _, pooled = O.decode_anchor(q, k, v, [T], scale)
+        idx = np.stack([[O.topk_select(pooled[0][h], kk) for h in range(cfg.Hkv)]])
+        t1 = time.perf_counter()
+        O.decode_reuse(qr, kr, vr, [T], idx, np.full((1, cfg.Hkv), kk), hm, scale)
+        t2 = time.perf_counter()
+        t_a += t1 - t0
+        t_r += t2 - t1
+    t_a /= steps
+    t_r /= steps
+    na = len(cfg.anchors)
+    dec_us = (na * t_a + (cfg.n_layers - na) * t_r) * cfg.B / cfg.n_layers * 1e6
+
+    pcfg = workload.PREFILL_16K
+    grp = workload.prefill_group(pcfg, 0, 0, 0)
+    G = pcfg.Hq // pcfg.Hkv
+    qg = np.zeros((G, pcfg.N, pcfg.d))
+    qg[:] = grp["q"].float().numpy()
+    kg = grp["k"].float().numpy()[None]
+    vg = grp["v"].float().numpy()[None]
+    tiles = [pcfg.N // pcfg.tile - 1, pcfg.N // pcfg.tile // 2]
+    t0 = time.perf_counter()
+    _, _, pooled = O.prefill_anchor(qg, kg, vg, scale, tile=pcfg.tile, tiles=tiles)
+    nt = pcfg.N // pcfg.tile
+    kmax = O.k_for_len(pcfg.N - pcfg.tile)
+    idx = np.full((nt, 1, kmax), -1)
+    idx_k = np.zeros((nt, 1), dtype=np.int64)
+    for t in tiles:
+        kt = O.k_for_len(pcfg.tile * t)
+        idx[t, 0, :kt] = O.topk_select(pooled[t, 0, : pcfg.tile * t], kt)
+        idx_k[t, 0] = kt
+    t1 = time.perf_counter()
+    O.prefill_reuse(qg, kg, vg, idx, idx_k, [0], scale, tile=pcfg.tile, tiles=tiles)
+    t2 = time.perf_counter()
+    # scale by causal pairs: sample tiles' pairs vs all tiles, and 1 of Hkv groups
+    tile_pairs = lambda t: pcfg.tile * pcfg.tile * t + pcfg.tile * (pcfg.tile + 1) // 2  # noqa: E731
+    all_pairs = sum(tile_pairs(t) for t in range(nt))
+    s_pairs = sum(tile_pairs(t) for t in tiles)
+    reuse_pairs = lambda t: pcfg.tile * O.k_for_len(pcfg.tile * t) + pcfg.tile * (pcfg.tile + 1) // 2  # noqa: E731
+    r_all = sum(reuse_pairs(t) for t in range(nt))
+    r_s = sum(reuse_pairs(t) for t in tiles)
+    pa_ms = (t1 - t0) * all_pairs / s_pairs * pcfg.Hkv * 1e3
+    pr_ms = (t2 - t1) * r_all / r_s * pcfg.Hkv * 1e3
+    na = len(pcfg.anchors)
+    pre_ms = (na * pa_ms + (pcfg.n_layers - na) * pr_ms) / pcfg.n_layers
+    sample = (f"decode: anchor+topk and one reuse layer for 1 of 16 sequences (T=32768), scaled to "
+              f"B=16 and the 5/27 anchor/reuse mix; prefill: tiles {tiles} of KV head 0 (anchor + "
+              f"reuse), scaled by causal key pairs to 128 tiles x 8 KV heads")
+    return dec_us, pre_ms, sample, cores, {"decode_anchor_s_per_seq": t_a,
+                                            "decode_reuse_s_per_seq": t_r,
+                                            "prefill_anchor_sample_s": t1 - t0,
+                                            "prefill_reuse_sample_s": t2 - t1}
+
+
+def run_reference(args, dist):
+    """--impl reference: the oracle, as it stands, on the host cores."""
+    if dist.rank != 0:
+        return
+    vals = []
+    cpu_sample(1)  # warm numpy / BLAS once regardless of W
+    for _ in range(max(args.warmup - 1, 0)):
+        cpu_sample(1)
+    res = None
+    for _ in range(args.steps):
+        res = cpu_sample(1)
+        vals.append(res[0])
+    dec_us = float(np.mean(vals))
+    _, pre_ms, sample, cores, _ = res
+    line = {"impl": "reference", "metric": METRIC, "value": dec_us, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dec_us * 32 / 1e3 + pre_ms * 4, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "decode_b16_t32768 + prefill_b1_n16384 (bounded oracle sample)",
+                       "prefill_ms_per_layer": pre_ms},
+            "cpu_baseline": {"value": dec_us, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": dec_us, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------------------
+def main():
+    args = parse()
+    dist = Dist()
+    if args.impl == "reference":
+        run_reference(args, dist)
+        dist.close()
+        return
+
+    from long_context_emitting_b200 import api, binding
+
+    binding.load()
+    dev = torch.device("cuda", dist.local)
+    torch.cuda.set_device(dev)
+    pk, pk_kind = peaks()
+    do_dec = args.only in ("all", "decode")
+    do_pre = args.only in ("all", "prefill")
+
+    dec = build_decode(dev, args.decode_layers) if do_dec else None
+    pre = build_prefill(dev) if do_pre else None
+    torch.cuda.synchronize()
+
+    def step(timer=None):
+        if dec:
+            decode_step(dec[1], dec[2], dec[3], dec[4], timer)
+        if pre:
+            prefill_step(pre[1], pre[2], pre[3], pre[4], timer)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if api.device_status() != 0:
+        raise RuntimeError("device status set during warm-up")
+
+    clocks = Clocks(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                    else int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[dist.local]))
+    timer = OpTimer()
+    dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record()
+    for _ in range(args.steps):
+        step(timer)
+    t_end.record()
+    torch.cuda.synchronize()
+    dist.barrier()
+    clk = clocks.stop()
+    timer.collect()
+    total_ms = dist.max(t_start.elapsed_time(t_end))
+    ms_per_step = total_ms / args.steps
+    N = dist.world
+
+    out = {"metric": METRIC, "unit": UNIT, "n_gpus": N, "steps": args.steps,
+           "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": False,
+           "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+           "data": "synthetic: seeded planted-heavy-key generator (no datasets or weights)"}
+    roofline = None
+    cfgd = {}
+    if dec:
+        cfg, sch = dec[0], dec[1]
+        L = sch.n_layers
+        n_anchor = sum(1 for l in range(L) if sch.is_anchor(l))
+        dec_ms = dist.max((timer.total_ms("dec_anchor") + timer.total_ms("dec_topk")
+                           + timer.total_ms("dec_reuse")) / args.steps)
+        us_layer = dec_ms * 1e3 / (L * N)
+        anchor_ms = timer.mean_ms("dec_anchor")
+        topk_ms = timer.mean_ms("dec_topk")
+        reuse_ms = timer.mean_ms("dec_reuse")
+        Hkv = cfg.Hkv
+        toks = sum(sch.lens)
+        anchor_bytes = toks * Hkv * (cfg.d * 2 * 2 + 4)            # K+V read, pooled write
+        reuse_bytes = sch.reuse_bytes_per_layer                      # gathered K+V rows
+        step_bytes = n_anchor * anchor_bytes + (L - n_anchor) * reuse_bytes
+        out["value"] = us_layer
+        out["decode"] = {
+            "us_per_layer": us_layer, "layers": L, "anchor_layers": n_anchor,
+            "anchor_us": anchor_ms * 1e3, "topk_us": topk_ms * 1e3, "reuse_us": reuse_ms * 1e3,
+            "anchor_hbm_gbs": anchor_bytes / (anchor_ms * 1e-3) / 1e9 if anchor_ms else None,
+            "reuse_hbm_gbs": reuse_bytes / (reuse_ms * 1e-3) / 1e9 if reuse_ms else None,
+            "step_hbm_gbs": step_bytes / (dec_ms * 1e-3) / 1e9 * N,
+            "reuse_over_anchor_layer_time": reuse_ms / anchor_ms if anchor_ms else None,
+            "reuse_over_anchor_time_per_token": ((reuse_ms / (sch.row_k.sum().item() / Hkv))
+                                                 / (anchor_ms / toks))
+            if anchor_ms and reuse_ms else None,
+        }
+        peak = pk["hbm_gbs"]
+        ach = anchor_bytes / (anchor_ms * 1e-3) / 1e9
+        roofline = {"bound": "hbm", "kernel": "decode anchor (split-K attention + pooled epilogue)",
+                    "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+                    "peak_source": f"{pk_kind} hbm_gbs", "traffic": None,
+                    "algorithmic_bytes_per_launch": anchor_bytes}
+        cfgd["decode"] = {"name": cfg.name, "B": cfg.B, "T": cfg.T, "layers": L,
+                          "anchors": list(cfg.anchors), "k": int(sch.k_max), "Hq": cfg.Hq,
+                          "Hkv": cfg.Hkv, "d": cfg.d}
+    if pre:
+        cfg, sch = pre[0], pre[1]
+        pre_ms = dist.max((timer.total_ms("pre_anchor") + timer.total_ms("pre_topk")
+                           + timer.total_ms("pre_reuse")) / args.steps)
+        pa = timer.mean_ms("pre_anchor")
+        pt = timer.mean_ms("pre_topk")
+        pr = timer.mean_ms("pre_reuse")
+        N_tok = cfg.N
+        flops_anchor = 4.0 * cfg.d * cfg.Hq * N_tok * (N_tok + 1) / 2
+        nt = N_tok // cfg.tile
+        from long_context_emitting_b200 import api as _api
+        reuse_pairs = sum(cfg.tile * _api.k_for_len(cfg.tile * t) + cfg.tile * (cfg.tile + 1) // 2
+                          for t in range(nt))
+        flops_reuse = 4.0 * cfg.d * cfg.Hq * reuse_pairs
+        out["prefill"] = {
+            "ms_per_layer": pre_ms / (sch.n_layers * N), "anchor_ms": pa, "topk_ms": pt,
+            "reuse_ms": pr,
+            "anchor_tflops": flops_anchor / (pa * 1e-3) / 1e12 if pa else None,
+            "reuse_tflops": flops_reuse / (pr * 1e-3) / 1e12 if pr else None,
+            "anchor_frac_of_bf16_peak": (flops_anchor / (pa * 1e-3) / 1e12) / pk["bf16_tflops"]
+            if pa else None,
+        }
+        cfgd["prefill"] = {"name": cfg.name, "B": cfg.B, "N": cfg.N, "layers": cfg.n_layers,
+                           "anchors": list(cfg.anchors), "tile": cfg.tile}
+        if not dec:
+            out["value"] = pre_ms / (sch.n_layers * N)
+            out["unit"] = "ms/layer"
+    from long_context_emitting_b200.schedule import launches_per_step
+    launches = launches_per_step(dec[1] if dec else None, pre[1] if pre else None) * args.steps
+    out["gpu_launches"] = launches
+    out["config"] = {"workload": "decode_b16_t32768 (32 layers) + prefill_b1_n16384 (4 layers)",
+                     **cfgd, "l2": "inputs larger than L2 (2.1 GB of KV per decode layer)",
+                     "parallelism": f"replicas x{N}"}
+    out["roofline"] = roofline
+    out["clocks"] = clk
+
+    if not args.no_e2e:
+        out["e2e"] = e2e(dec, pre, args, dist)
+    if not args.no_cpu and dist.rank == 0:
+        dus, pms, sample, cores, raw = cpu_sample(1)
+        out["cpu_baseline"] = {"value": dus, "unit": UNIT, "cores": cores, "kind": "oracle",
+                               "sample": sample, "prefill_ms_per_layer": pms, "raw": raw}
+    if dist.rank == 0:
+        print(json.dumps(out), flush=True)
+    dist.close()
+
+
+def e2e(dec, pre, args, dist):
+    """Same metric through the public API with pinned host buffers: every step
+    copies its new queries (decode; the KV cache is device-resident state) or
+    its q/k/v (prefill) host->device and reads the outputs back."""
+    h2d = d2h = 0
+    res = {"unit": UNIT}
+    if dec:
+        cfg, sch, layers, maps, outs = dec
+        L = sch.n_layers
+        q_host = torch.stack([layers[l]["q"] for l in range(L)]).cpu().pin_memory()
+        o_host = torch.empty_like(q_host).pin_memory()
+        q_dev = [layers[l]["q"] for l in range(L)]
+        h2d += q_host.numel() * 2
+        d2h += o_host.numel() * 2
+
+        def dstep():
+            for l in range(L):
+                q_dev[l].copy_(q_host[l], non_blocking=True)
+            decode_step(sch, layers, maps, outs)
+            for l in range(L):
+                o_host[l].copy_(outs[l], non_blocking=True)
+
+        for _ in range(2):
+            dstep()
+        torch.cuda.synchronize()
+        dist.barrier()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(args.steps):
+            dstep()
+        e.record()
+        torch.cuda.synchronize()
+        ms = dist.max(s.elapsed_time(e)) / args.steps
+        res["value"] = ms * 1e3 / (L * dist.world)
+    if pre:
+        cfg, sch, layers, maps, outs = pre
+        L = sch.n_layers
+        hq = [{n: layers[l][n].cpu().pin_memory() for n in ("q", "k", "v")} for l in range(L)]
+        ho = [torch.empty_like(hq[l]["q"]).pin_memory() for l in range(L)]
+        for l in range(L):
+            h2d += sum(t.numel() * 2 for t in hq[l].values())
+            d2h += ho[l].numel() * 2
+
+        def pstep():
+            for l in range(L):
+                for n in ("q", "k", "v"):
+                    layers[l][n].copy_(hq[l][n], non_blocking=True)
+            prefill_step(sch, layers, maps, outs)
+            for l in range(L):
+                ho[l].copy_(outs[l], non_blocking=True)
+
+        pstep()
+        torch.cuda.synchronize()
+        dist.barrier()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(args.steps):
+            pstep()
+        e.record()
+        torch.cuda.synchronize()
+        pms = dist.max(s.elapsed_time(e)) / args.steps
+        res["prefill_ms_per_layer"] = pms / (L * dist.world)
+        if not dec:
+            res["value"] = res["prefill_ms_per_layer"]
+            res["unit"] = "ms/layer"
+    res["h2d_bytes_per_step"] = h2d
+    res["d2h_bytes_per_step"] = d2h
+    return res
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,178 @@
+/*
+ * kascade.h -- C ABI of the Kascade attention hot path on NVIDIA B200 (sm_100a).
+ *
+ * Kascade (arXiv 2512.16391) splits a model's layers into anchor layers, which
+ * run dense attention and take the Top-k keys of the post-softmax
+ * distribution, and reuse layers, which attend only to the keys an anchor
+ * chose, per key head through a head-remap table.
+ * Sources, cited by page and section:
+ *   [explainer] "論文解説: Kascade — レイヤー間スパーシティ再利用による実用的長文脈LLM推論高速化"
+ *               (0h-n0.github.io), sections under 技術的詳細 and 実装のポイント;
+ *   [abstract]  the arXiv abstract (fugumt.com listing of 2512.16391v1).
+ *
+ * General rules (every entry point):
+ *   - Every pointer argument is a DEVICE pointer owned by the caller; the library
+ *     never allocates, frees or keeps a pointer after the call returns.  Scratch
+ *     memory is passed in as `ws` of `ws_bytes` (query the size first).
+ *   - bf16 tensors are passed as uint16_t bit patterns (IEEE bfloat16).
+ *   - Every base pointer must be 16-byte aligned; every row stride named below is
+ *     in elements and must keep rows 16-byte aligned.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is enqueued
+ *     asynchronously; the return value reports only what the host can check before
+ *     launching (arguments, shapes, workspace size, launch errors).
+ *   - Errors found by the kernels themselves (an index, head-map entry or length
+ *     out of range, a NaN score) never fault: the offending element is skipped, and
+ *     a sticky per-device status word is set; read it with kascade_get_device_status.
+ *   - Supported shapes: head_dim d == 128, Hq % Hkv == 0, group size Hq/Hkv <= 8,
+ *     prefill query tile fixed at 128 tokens, prefill length a multiple of 128.
+ *   - Returned status codes are the kascade_status values below; no C++ exception
+ *     crosses this boundary.
+ */
+#ifndef KASCADE_H_
+#define KASCADE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KASCADE_OK = 0,
+  KASCADE_ERR_INVALID_ARG = 1,        /* NULL/misaligned pointer, negative size, k > length ... */
+  KASCADE_ERR_UNSUPPORTED_SHAPE = 2,  /* d != 128, group > 8, prefill N not a multiple of 128 */
+  KASCADE_ERR_WORKSPACE_TOO_SMALL = 3,
+  KASCADE_ERR_CUDA = 4,               /* a launch or CUDA runtime call failed */
+  KASCADE_ERR_BAD_INDEX = 5,          /* device side: index / head map / length out of range */
+  KASCADE_ERR_NONFINITE = 6           /* device side: NaN in a Top-k score row */
+} kascade_status;
+
+/* Attention shape shared by all calls.  B = batch, Hq = query heads,
+ * Hkv = key/value heads (GQA group G = Hq / Hkv), d = head dim (128). */
+typedef struct {
+  int32_t B, Hq, Hkv, d;
+} kascade_shape;
+
+/* ------------------------------------------------------------------------- */
+/* Top-k size rule.  [explainer] 技術的詳細 › Top-k設定, k equation:
+ * k = min(max(0.1·n, 128), n) with 0.1·n rounded half up, i.e.
+ * min(max((n + 5) / 10, 128), n) in integer arithmetic.  n < 0 returns 0. */
+int32_t kascade_k_for_len(int32_t n);
+
+/* ------------------------------------------------------------------------- */
+/* Decode anchor layer.  [explainer] 技術的詳細 › アンカーレイヤーと再利用レイヤー (full attention
+ * in anchor layers, Top-k from the post-softmax distribution) and › ヘッドリマッピング (one
+ * index set per key head under GQA).
+ *
+ * For sequence b, KV head h and each query head g of group h (g in [G·h, G·h+G)):
+ *   s_{g,t} = scale · q[b,g,:] · K[b,h,t,:]       for t < T_b = seq_len[b]
+ *   out[b,g,:] = sum_t softmax_t(s_g)_t · V[b,h,t,:]
+ *   lse[b,g]   = log sum_t exp(s_{g,t})           (natural log)
+ *   pooled[b,h,t] = (1/G) · sum_g exp(s_{g,t} - lse[b,g])   (mean post-softmax probability)
+ *
+ *   q       bf16 [B, Hq, d]
+ *   k, v    bf16 caches; sequence b is a contiguous [Hkv, T_b, d] block starting at
+ *           element kv_off[b] of k (and of v)
+ *   kv_off  int64 [B] element offsets (multiples of 8); seq_len int32 [B], 0 <= T_b <= max_T
+ *   max_T   host-side upper bound of seq_len (sizes the grid and the workspace)
+ *   out     bf16 [B, Hq, d]; lse fp32 [B, Hq] (may be NULL)
+ *   pooled  fp32 [B, Hkv, ld_pooled], ld_pooled >= max_T, ld_pooled % 4 == 0; entries at
+ *           t >= T_b are left untouched
+ *   ws      scratch of at least kascade_decode_anchor_workspace_bytes(s, max_T) bytes
+ * A sequence with T_b == 0 gets out = 0 and lse = -inf. */
+size_t kascade_decode_anchor_workspace_bytes(kascade_shape s, int32_t max_T);
+int kascade_decode_anchor(kascade_shape s, const uint16_t* q, const uint16_t* k,
+                          const uint16_t* v, const int64_t* kv_off, const int32_t* seq_len,
+                          int32_t max_T, float scale, uint16_t* out, float* lse,
+                          float* pooled, int64_t ld_pooled, void* ws, size_t ws_bytes,
+                          void* stream);
+
+/* ------------------------------------------------------------------------- */
+/* Row-wise Top-k select.  [explainer] 技術的詳細 › アンカーレイヤーと再利用レイヤー (exact Top-k
+ * indices in anchor layers) and › Top-k設定 (k).  Ties are broken toward the lower index;
+ * -0.0 equals +0.0; the selected indices are written in ascending order.
+ *
+ *   scores   fp32 [rows, ld]; row r uses its first row_len[r] entries
+ *   row_len  int32 [rows], 0 <= row_len[r] <= ld
+ *   row_k    int32 [rows], 0 <= row_k[r] <= min(row_len[r], k_max)
+ *   idx_out  int32 [rows, k_max]; entries past row_k[r] are set to -1
+ *   ws       scratch of kascade_topk_workspace_bytes(rows, ld) bytes (may be 0 / NULL)
+ * A NaN in a row sets KASCADE_ERR_NONFINITE on the device (that row's output is
+ * unspecified); a bad row_len / row_k sets KASCADE_ERR_BAD_INDEX and writes -1s. */
+size_t kascade_topk_workspace_bytes(int32_t rows, int64_t ld);
+int kascade_topk(const float* scores, int32_t rows, int64_t ld, const int32_t* row_len,
+                 const int32_t* row_k, int32_t k_max, int32_t* idx_out, void* ws,
+                 size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------- */
+/* Decode reuse layer.  [explainer] アンカーレイヤーと再利用レイヤー (reuse layers attend only to
+ * the keys the preceding anchor selected) and ヘッドリマッピング (reuse key head h takes the
+ * indices of anchor key head head_map[h]).  The softmax is renormalised over the set.
+ *
+ * For sequence b, reuse KV head h, a = head_map[h], J = idx[b, a, 0 : idx_k[b·Hkv + a]]:
+ *   out[b,g,:] = sum_{j in J} softmax_J(scale · q[b,g,:]·K[b,h,j,:])_j · V[b,h,j,:]
+ *
+ *   q, k, v, kv_off, seq_len   as in kascade_decode_anchor
+ *   idx      int32 [B, Hkv, k_max]   anchor indices, each in [0, T_b)
+ *   idx_k    int32 [B·Hkv]           valid count per anchor row, <= k_max
+ *   head_map int32 [Hkv]             values in [0, Hkv)
+ *   out bf16 [B, Hq, d]; lse fp32 [B, Hq] (may be NULL)
+ *   ws       scratch of kascade_decode_reuse_workspace_bytes(s, k_max) bytes
+ * Out-of-range indices are skipped (status KASCADE_ERR_BAD_INDEX). */
+size_t kascade_decode_reuse_workspace_bytes(kascade_shape s, int32_t k_max);
+int kascade_decode_reuse(kascade_shape s, const uint16_t* q, const uint16_t* k,
+                         const uint16_t* v, const int64_t* kv_off, const int32_t* seq_len,
+                         const int32_t* idx, const int32_t* idx_k, int32_t k_max,
+                         const int32_t* head_map, float scale, uint16_t* out, float* lse,
+                         void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------- */
+/* Prefill anchor layer.  [explainer] 主要な貢献 (tile-level post-softmax pooling in
+ * prefill), 実装のポイント (128-query tiles in prefill), アンカーレイヤーと再利用レイヤー.
+ *
+ * Causal attention over N tokens: query i sees keys j <= i.  For query tile t
+ * (queries [128t, 128t+128)) and KV head h:
+ *   pooled[b,t,h,j] = 1/(128·G) · sum_{i in tile t} sum_{g in group h}
+ *                      exp(s_{g,i,j} - lse[b,g,i])          for j < 128t
+ *
+ *   q bf16 [B, Hq, N, d]; k, v bf16 [B, Hkv, N, d]
+ *   out bf16 [B, Hq, N, d]; lse fp32 [B, Hq, N] (required: it is the pooling normaliser)
+ *   pooled fp32 [B, N/128, Hkv, N]; entries at j >= 128t are left untouched
+ *   ws scratch of kascade_prefill_anchor_workspace_bytes(s, N) bytes */
+size_t kascade_prefill_anchor_workspace_bytes(kascade_shape s, int32_t N);
+int kascade_prefill_anchor(kascade_shape s, int32_t N, const uint16_t* q, const uint16_t* k,
+                           const uint16_t* v, float scale, uint16_t* out, float* lse,
+                           float* pooled, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------- */
+/* Prefill reuse layer.  [explainer] アンカーレイヤーと再利用レイヤー, ヘッドリマッピング,
+ * 実装のポイント (128-query tiles).  Query i of tile t in reuse KV head h attends to
+ *   J_t = idx[b, t, head_map[h], 0 : idx_k[(b·n_tiles + t)·Hkv + head_map[h]]]   (all < 128t)
+ * together with its own diagonal block, causally (keys 128t <= j <= i); softmax over
+ * that set.
+ *
+ *   q, k, v as in kascade_prefill_anchor
+ *   idx int32 [B, N/128, Hkv, k_max]; idx_k int32 [B·(N/128)·Hkv]; head_map int32 [Hkv]
+ *   out bf16 [B, Hq, N, d]; lse fp32 [B, Hq, N] (may be NULL)
+ *   ws scratch of kascade_prefill_reuse_workspace_bytes(s, N, k_max) bytes */
+size_t kascade_prefill_reuse_workspace_bytes(kascade_shape s, int32_t N, int32_t k_max);
+int kascade_prefill_reuse(kascade_shape s, int32_t N, const uint16_t* q, const uint16_t* k,
+                          const uint16_t* v, const int32_t* idx, const int32_t* idx_k,
+                          int32_t k_max, const int32_t* head_map, float scale, uint16_t* out,
+                          float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------- */
+/* Waits for `stream`, then returns and clears the sticky device status of the
+ * current device: KASCADE_OK, or the first of KASCADE_ERR_BAD_INDEX /
+ * KASCADE_ERR_NONFINITE that a kernel recorded (KASCADE_ERR_CUDA if the wait fails). */
+int kascade_get_device_status(void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* kascade_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KASCADE_H_ */

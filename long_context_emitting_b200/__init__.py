@@ -1,0 +1,14 @@
+"""Kascade hot path (head-aware Top-k sparse attention with cross-layer index
+reuse) on NVIDIA B200: a C-ABI CUDA library (libkascade.so, include/kascade.h)
+with a thin PyTorch/ctypes binding.
+
+Modules:
+  binding   -- ctypes declarations of the C entry points (marshalling only)
+  api       -- tensor-level calls of the same names on the current CUDA stream
+  schedule  -- anchor / Top-k / reuse layer schedule with preallocated buffers
+  workload  -- seeded synthetic inputs shaped like the evaluated workloads
+  build     -- nvcc build of libkascade.so for sm_100a
+"""
+from . import api, binding, schedule, workload  # noqa: F401
+
+__all__ = ["api", "binding", "schedule", "workload"]

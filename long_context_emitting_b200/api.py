@@ -1,0 +1,187 @@
+"""Tensor-level entry points: PyTorch CUDA tensors in, C-ABI calls out.
+
+Each function checks dtypes/devices/contiguity, allocates outputs and the
+workspace with PyTorch when the caller passes none, and calls the entry point
+of the same name in libkascade.so on the current CUDA stream.  All arithmetic
+runs in the library's kernels; CPU tensors are rejected.
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional
+
+import torch
+
+from . import binding
+from .binding import Shape, check
+
+HEAD_DIM = 128
+TILE = 128
+
+
+def _lib():
+    return binding.load()
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _need_cuda(name: str, t: torch.Tensor, dtype: torch.dtype) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (the library has no CPU path)")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _bits(t: torch.Tensor) -> torch.Tensor:
+    return t.view(torch.int16) if t.dtype == torch.bfloat16 else t
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def k_for_len(n: int) -> int:
+    """Top-k size for a context of n keys (the library's rule)."""
+    return int(_lib().kascade_k_for_len(int(n)))
+
+
+def device_status(stream: Optional[int] = None) -> int:
+    """Wait for the stream and return/clear the sticky device status code."""
+    return int(_lib().kascade_get_device_status(_stream() if stream is None else stream))
+
+
+def workspace(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device)
+
+
+# ---------------------------------------------------------------- decode ----
+def decode_anchor_workspace_bytes(B, Hq, Hkv, max_T) -> int:
+    return int(_lib().kascade_decode_anchor_workspace_bytes(Shape(B, Hq, Hkv, HEAD_DIM), max_T))
+
+
+def decode_anchor(q, k, v, kv_off, seq_len, max_T: int, scale: float, Hkv: int,
+                  out=None, lse=None, pooled=None, ld_pooled: Optional[int] = None, ws=None):
+    """Dense decode attention + GQA-pooled probabilities (kascade_decode_anchor)."""
+    B, Hq, d = q.shape
+    _need_cuda("q", q, torch.bfloat16)
+    _need_cuda("k", k, torch.bfloat16)
+    _need_cuda("v", v, torch.bfloat16)
+    _need_cuda("kv_off", kv_off, torch.int64)
+    _need_cuda("seq_len", seq_len, torch.int32)
+    dev = q.device
+    if ld_pooled is None:
+        ld_pooled = (max_T + 3) // 4 * 4
+    out = torch.empty(B, Hq, d, dtype=torch.bfloat16, device=dev) if out is None else out
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=dev) if lse is None else lse
+    pooled = torch.empty(B, Hkv, ld_pooled, dtype=torch.float32, device=dev) if pooled is None else pooled
+    shape = Shape(B, Hq, Hkv, d)
+    need = _lib().kascade_decode_anchor_workspace_bytes(shape, max_T)
+    ws = workspace(need, dev) if ws is None else ws
+    rc = _lib().kascade_decode_anchor(shape, _ptr(q), _ptr(k), _ptr(v), _ptr(kv_off), _ptr(seq_len),
+                                      int(max_T), float(scale), _ptr(out), _ptr(lse), _ptr(pooled),
+                                      int(ld_pooled), _ptr(ws), ws.numel(), _stream())
+    check(rc, "kascade_decode_anchor")
+    return out, lse, pooled
+
+
+def decode_reuse_workspace_bytes(B, Hq, Hkv, k_max) -> int:
+    return int(_lib().kascade_decode_reuse_workspace_bytes(Shape(B, Hq, Hkv, HEAD_DIM), k_max))
+
+
+def decode_reuse(q, k, v, kv_off, seq_len, idx, idx_k, head_map, scale: float, Hkv: int,
+                 out=None, lse=None, ws=None):
+    """Sparse decode attention over anchor indices via a head map (kascade_decode_reuse)."""
+    B, Hq, d = q.shape
+    for name, t, dt in (("q", q, torch.bfloat16), ("k", k, torch.bfloat16), ("v", v, torch.bfloat16),
+                        ("kv_off", kv_off, torch.int64), ("seq_len", seq_len, torch.int32),
+                        ("idx", idx, torch.int32), ("idx_k", idx_k, torch.int32),
+                        ("head_map", head_map, torch.int32)):
+        _need_cuda(name, t, dt)
+    k_max = idx.shape[-1]
+    dev = q.device
+    out = torch.empty(B, Hq, d, dtype=torch.bfloat16, device=dev) if out is None else out
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=dev) if lse is None else lse
+    shape = Shape(B, Hq, Hkv, d)
+    need = _lib().kascade_decode_reuse_workspace_bytes(shape, k_max)
+    ws = workspace(need, dev) if ws is None else ws
+    rc = _lib().kascade_decode_reuse(shape, _ptr(q), _ptr(k), _ptr(v), _ptr(kv_off), _ptr(seq_len),
+                                     _ptr(idx), _ptr(idx_k), int(k_max), _ptr(head_map),
+                                     float(scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                     _stream())
+    check(rc, "kascade_decode_reuse")
+    return out, lse
+
+
+# ------------------------------------------------------------------ topk ----
+def topk(scores, row_len, row_k, k_max: int, out=None):
+    """Row-wise Top-k (ties to lower index, ascending output; tail = -1)."""
+    _need_cuda("scores", scores, torch.float32)
+    _need_cuda("row_len", row_len, torch.int32)
+    _need_cuda("row_k", row_k, torch.int32)
+    ld = scores.shape[-1]
+    rows = scores.numel() // ld if ld else 0
+    out = torch.empty(rows, k_max, dtype=torch.int32, device=scores.device) if out is None else out
+    rc = _lib().kascade_topk(_ptr(scores), int(rows), int(ld), _ptr(row_len), _ptr(row_k),
+                             int(k_max), _ptr(out), None, 0, _stream())
+    check(rc, "kascade_topk")
+    return out
+
+
+# --------------------------------------------------------------- prefill ----
+def prefill_anchor_workspace_bytes(B, Hq, Hkv, N) -> int:
+    return int(_lib().kascade_prefill_anchor_workspace_bytes(Shape(B, Hq, Hkv, HEAD_DIM), N))
+
+
+def prefill_anchor(q, k, v, scale: float, out=None, lse=None, pooled=None, ws=None):
+    """Dense causal prefill attention + tile-pooled probabilities (kascade_prefill_anchor)."""
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need_cuda(name, t, torch.bfloat16)
+    dev = q.device
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty(B, Hq, N, dtype=torch.float32, device=dev) if lse is None else lse
+    if pooled is None:
+        pooled = torch.empty(B, N // TILE, Hkv, N, dtype=torch.float32, device=dev)
+    shape = Shape(B, Hq, Hkv, d)
+    need = _lib().kascade_prefill_anchor_workspace_bytes(shape, N)
+    ws = workspace(need, dev) if ws is None else ws
+    rc = _lib().kascade_prefill_anchor(shape, int(N), _ptr(q), _ptr(k), _ptr(v), float(scale),
+                                       _ptr(out), _ptr(lse), _ptr(pooled), _ptr(ws), ws.numel(),
+                                       _stream())
+    check(rc, "kascade_prefill_anchor")
+    return out, lse, pooled
+
+
+def prefill_reuse_workspace_bytes(B, Hq, Hkv, N, k_max) -> int:
+    return int(_lib().kascade_prefill_reuse_workspace_bytes(Shape(B, Hq, Hkv, HEAD_DIM), N, k_max))
+
+
+def prefill_reuse(q, k, v, idx, idx_k, head_map, scale: float, out=None, lse=None, ws=None):
+    """Sparse causal prefill attention over tile indices + diagonal (kascade_prefill_reuse)."""
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    for name, t, dt in (("q", q, torch.bfloat16), ("k", k, torch.bfloat16), ("v", v, torch.bfloat16),
+                        ("idx", idx, torch.int32), ("idx_k", idx_k, torch.int32),
+                        ("head_map", head_map, torch.int32)):
+        _need_cuda(name, t, dt)
+    k_max = idx.shape[-1]
+    dev = q.device
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty(B, Hq, N, dtype=torch.float32, device=dev) if lse is None else lse
+    shape = Shape(B, Hq, Hkv, d)
+    need = _lib().kascade_prefill_reuse_workspace_bytes(shape, N, k_max)
+    ws = workspace(need, dev) if ws is None else ws
+    rc = _lib().kascade_prefill_reuse(shape, int(N), _ptr(q), _ptr(k), _ptr(v), _ptr(idx),
+                                      _ptr(idx_k), int(k_max), _ptr(head_map), float(scale),
+                                      _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream())
+    check(rc, "kascade_prefill_reuse")
+    return out, lse
+
+
+def default_scale(d: int = HEAD_DIM) -> float:
+    return 1.0 / math.sqrt(d)

@@ -1,0 +1,240 @@
+// C ABI of the Kascade hot path: argument checks, workspace sizing, the sticky
+// device status word, and dispatch to the kernel launchers.  See
+// include/kascade.h for the contract of every entry point.
+#include "../../include/kascade.h"
+#include "common.cuh"
+#include "internal.h"
+
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+namespace kascade {
+__device__ unsigned int g_device_status = 0u;
+}
+
+using namespace kascade;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+unsigned* device_status_ptr() {
+  static unsigned* cache[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  if (!cache[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+    cache[dev] = static_cast<unsigned*>(p);
+  }
+  return cache[dev];
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_shape(const kascade_shape& s) {
+  if (s.B < 0 || s.Hq <= 0 || s.Hkv <= 0) return KASCADE_ERR_INVALID_ARG;
+  if (s.d != kHeadDim) return KASCADE_ERR_UNSUPPORTED_SHAPE;
+  if (s.Hq % s.Hkv) return KASCADE_ERR_UNSUPPORTED_SHAPE;
+  const int G = s.Hq / s.Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return KASCADE_ERR_UNSUPPORTED_SHAPE;
+  return KASCADE_OK;
+}
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? KASCADE_OK : KASCADE_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int32_t kascade_k_for_len(int32_t n) {
+  if (n <= 0) return 0;
+  const int32_t tenth = (int32_t)(((int64_t)n + 5) / 10);
+  const int32_t k = tenth > 128 ? tenth : 128;
+  return k < n ? k : n;
+}
+
+const char* kascade_status_string(int status) {
+  switch (status) {
+    case KASCADE_OK: return "KASCADE_OK";
+    case KASCADE_ERR_INVALID_ARG: return "KASCADE_ERR_INVALID_ARG";
+    case KASCADE_ERR_UNSUPPORTED_SHAPE: return "KASCADE_ERR_UNSUPPORTED_SHAPE";
+    case KASCADE_ERR_WORKSPACE_TOO_SMALL: return "KASCADE_ERR_WORKSPACE_TOO_SMALL";
+    case KASCADE_ERR_CUDA: return "KASCADE_ERR_CUDA";
+    case KASCADE_ERR_BAD_INDEX: return "KASCADE_ERR_BAD_INDEX";
+    case KASCADE_ERR_NONFINITE: return "KASCADE_ERR_NONFINITE";
+    default: return "KASCADE_ERR_UNKNOWN";
+  }
+}
+
+int kascade_get_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return KASCADE_ERR_CUDA;
+  unsigned v = 0u;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v)) != cudaSuccess) return KASCADE_ERR_CUDA;
+  const unsigned zero = 0u;
+  if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero)) != cudaSuccess) return KASCADE_ERR_CUDA;
+  if (v & kStatusBadIndex) return KASCADE_ERR_BAD_INDEX;
+  if (v & kStatusNonFinite) return KASCADE_ERR_NONFINITE;
+  return KASCADE_OK;
+}
+
+// ------------------------------------------------------------------ decode --
+size_t kascade_decode_anchor_workspace_bytes(kascade_shape s, int32_t max_T) {
+  if (check_shape(s) != KASCADE_OK || max_T < 0) return 0;
+  return decode_workspace_bytes(s.B, s.Hkv, s.Hq / s.Hkv, max_T, true);
+}
+
+int kascade_decode_anchor(kascade_shape s, const uint16_t* q, const uint16_t* k,
+                          const uint16_t* v, const int64_t* kv_off, const int32_t* seq_len,
+                          int32_t max_T, float scale, uint16_t* out, float* lse,
+                          float* pooled, int64_t ld_pooled, void* ws, size_t ws_bytes,
+                          void* stream) {
+  int rc = check_shape(s);
+  if (rc) return rc;
+  if (max_T < 0 || ld_pooled < max_T || (ld_pooled & 3) || !std::isfinite(scale))
+    return KASCADE_ERR_INVALID_ARG;
+  if (s.B == 0) return KASCADE_OK;
+  if (!q || !k || !v || !kv_off || !seq_len || !out || !pooled || !ws) return KASCADE_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(pooled) ||
+      !aligned16(ws) || (lse && !aligned16(lse)) || ((uintptr_t)kv_off & 7) || ((uintptr_t)seq_len & 3))
+    return KASCADE_ERR_INVALID_ARG;
+  if (ws_bytes < kascade_decode_anchor_workspace_bytes(s, max_T)) return KASCADE_ERR_WORKSPACE_TOO_SMALL;
+  DecodeParams p = {};
+  p.B = s.B; p.Hq = s.Hq; p.Hkv = s.Hkv; p.G = s.Hq / s.Hkv;
+  p.q = q; p.k = k; p.v = v; p.kv_off = kv_off; p.seq_len = seq_len; p.max_T = max_T;
+  p.scale = scale; p.out = out; p.lse = lse; p.pooled = pooled; p.ld_pooled = ld_pooled;
+  p.ws = ws;
+  p.status = device_status_ptr();
+  if (!p.status) return KASCADE_ERR_CUDA;
+  return from_cuda(launch_decode_anchor(p, static_cast<cudaStream_t>(stream)));
+}
+
+size_t kascade_decode_reuse_workspace_bytes(kascade_shape s, int32_t k_max) {
+  if (check_shape(s) != KASCADE_OK || k_max < 0) return 0;
+  return decode_workspace_bytes(s.B, s.Hkv, s.Hq / s.Hkv, k_max, false);
+}
+
+int kascade_decode_reuse(kascade_shape s, const uint16_t* q, const uint16_t* k,
+                         const uint16_t* v, const int64_t* kv_off, const int32_t* seq_len,
+                         const int32_t* idx, const int32_t* idx_k, int32_t k_max,
+                         const int32_t* head_map, float scale, uint16_t* out, float* lse,
+                         void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_shape(s);
+  if (rc) return rc;
+  if (k_max < 0 || !std::isfinite(scale)) return KASCADE_ERR_INVALID_ARG;
+  if (s.B == 0) return KASCADE_OK;
+  if (!q || !k || !v || !kv_off || !seq_len || !idx || !idx_k || !head_map || !out || !ws)
+    return KASCADE_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(ws) ||
+      (lse && !aligned16(lse)) || ((uintptr_t)kv_off & 7) || ((uintptr_t)seq_len & 3) ||
+      ((uintptr_t)idx & 3) || ((uintptr_t)idx_k & 3) || ((uintptr_t)head_map & 3))
+    return KASCADE_ERR_INVALID_ARG;
+  if (ws_bytes < kascade_decode_reuse_workspace_bytes(s, k_max)) return KASCADE_ERR_WORKSPACE_TOO_SMALL;
+  DecodeParams p = {};
+  p.B = s.B; p.Hq = s.Hq; p.Hkv = s.Hkv; p.G = s.Hq / s.Hkv;
+  p.q = q; p.k = k; p.v = v; p.kv_off = kv_off; p.seq_len = seq_len;
+  p.max_T = 0x7fffffff;  // index validity is checked against each seq_len
+  p.idx = idx; p.idx_k = idx_k; p.head_map = head_map; p.k_max = k_max;
+  p.scale = scale; p.out = out; p.lse = lse; p.ws = ws;
+  p.status = device_status_ptr();
+  if (!p.status) return KASCADE_ERR_CUDA;
+  return from_cuda(launch_decode_reuse(p, static_cast<cudaStream_t>(stream)));
+}
+
+// -------------------------------------------------------------------- topk --
+size_t kascade_topk_workspace_bytes(int32_t rows, int64_t ld) {
+  (void)rows;
+  (void)ld;
+  return 0;
+}
+
+int kascade_topk(const float* scores, int32_t rows, int64_t ld, const int32_t* row_len,
+                 const int32_t* row_k, int32_t k_max, int32_t* idx_out, void* ws,
+                 size_t ws_bytes, void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  if (rows < 0 || ld < 0 || k_max < 0) return KASCADE_ERR_INVALID_ARG;
+  if (rows == 0) return KASCADE_OK;
+  if (!scores || !row_len || !row_k || (k_max > 0 && !idx_out)) return KASCADE_ERR_INVALID_ARG;
+  if (!aligned16(scores) || (ld & 3) || ((uintptr_t)row_len & 3) || ((uintptr_t)row_k & 3) ||
+      ((uintptr_t)idx_out & 3))
+    return KASCADE_ERR_INVALID_ARG;
+  unsigned* st = device_status_ptr();
+  if (!st) return KASCADE_ERR_CUDA;
+  return from_cuda(launch_topk(scores, rows, ld, row_len, row_k, k_max, idx_out, st,
+                               static_cast<cudaStream_t>(stream)));
+}
+
+// ----------------------------------------------------------------- prefill --
+static int check_prefill(const kascade_shape& s, int32_t N) {
+  int rc = check_shape(s);
+  if (rc) return rc;
+  if (N < 0) return KASCADE_ERR_INVALID_ARG;
+  if (N % 128) return KASCADE_ERR_UNSUPPORTED_SHAPE;
+  return KASCADE_OK;
+}
+
+size_t kascade_prefill_anchor_workspace_bytes(kascade_shape s, int32_t N) {
+  if (check_prefill(s, N) != KASCADE_OK) return 0;
+  return prefill_anchor_workspace_bytes(s.B, s.Hq, s.Hkv, N);
+}
+
+int kascade_prefill_anchor(kascade_shape s, int32_t N, const uint16_t* q, const uint16_t* k,
+                           const uint16_t* v, float scale, uint16_t* out, float* lse,
+                           float* pooled, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_prefill(s, N);
+  if (rc) return rc;
+  if (!std::isfinite(scale)) return KASCADE_ERR_INVALID_ARG;
+  if (s.B == 0 || N == 0) return KASCADE_OK;
+  const size_t need = kascade_prefill_anchor_workspace_bytes(s, N);
+  if (!q || !k || !v || !out || !lse || !pooled || (need && !ws)) return KASCADE_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse) ||
+      !aligned16(pooled) || (ws && !aligned16(ws)))
+    return KASCADE_ERR_INVALID_ARG;
+  if (ws_bytes < need) return KASCADE_ERR_WORKSPACE_TOO_SMALL;
+  PrefillParams p = {};
+  p.B = s.B; p.Hq = s.Hq; p.Hkv = s.Hkv; p.G = s.Hq / s.Hkv; p.N = N;
+  p.q = q; p.k = k; p.v = v; p.scale = scale; p.out = out; p.lse = lse; p.pooled = pooled;
+  p.ws = ws;
+  p.status = device_status_ptr();
+  if (!p.status) return KASCADE_ERR_CUDA;
+  cudaError_t e = launch_prefill_anchor(p, static_cast<cudaStream_t>(stream));
+  if (e == cudaErrorNotSupported) return KASCADE_ERR_UNSUPPORTED_SHAPE;
+  return from_cuda(e);
+}
+
+size_t kascade_prefill_reuse_workspace_bytes(kascade_shape s, int32_t N, int32_t k_max) {
+  if (check_prefill(s, N) != KASCADE_OK || k_max < 0) return 0;
+  return prefill_reuse_workspace_bytes(s.B, s.Hq, s.Hkv, N, k_max);
+}
+
+int kascade_prefill_reuse(kascade_shape s, int32_t N, const uint16_t* q, const uint16_t* k,
+                          const uint16_t* v, const int32_t* idx, const int32_t* idx_k,
+                          int32_t k_max, const int32_t* head_map, float scale, uint16_t* out,
+                          float* lse, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_prefill(s, N);
+  if (rc) return rc;
+  if (k_max < 0 || !std::isfinite(scale)) return KASCADE_ERR_INVALID_ARG;
+  if (s.B == 0 || N == 0) return KASCADE_OK;
+  const size_t need = kascade_prefill_reuse_workspace_bytes(s, N, k_max);
+  if (!q || !k || !v || !idx || !idx_k || !head_map || !out || (need && !ws))
+    return KASCADE_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      (lse && !aligned16(lse)) || (ws && !aligned16(ws)) || ((uintptr_t)idx & 3) ||
+      ((uintptr_t)idx_k & 3) || ((uintptr_t)head_map & 3))
+    return KASCADE_ERR_INVALID_ARG;
+  if (ws_bytes < need) return KASCADE_ERR_WORKSPACE_TOO_SMALL;
+  PrefillParams p = {};
+  p.B = s.B; p.Hq = s.Hq; p.Hkv = s.Hkv; p.G = s.Hq / s.Hkv; p.N = N;
+  p.q = q; p.k = k; p.v = v; p.idx = idx; p.idx_k = idx_k; p.head_map = head_map;
+  p.k_max = k_max; p.scale = scale; p.out = out; p.lse = lse; p.ws = ws;
+  p.status = device_status_ptr();
+  if (!p.status) return KASCADE_ERR_CUDA;
+  cudaError_t e = launch_prefill_reuse(p, static_cast<cudaStream_t>(stream));
+  if (e == cudaErrorNotSupported) return KASCADE_ERR_UNSUPPORTED_SHAPE;
+  return from_cuda(e);
+}
+
+}  // extern "C"

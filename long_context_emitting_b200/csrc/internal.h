@@ -1,0 +1,75 @@
+// Internal launch interface between the C-ABI layer (api.cu) and the kernel
+// translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace kascade {
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ---------------------------------------------------------------- decode ----
+struct DecodeParams {
+  int B, Hq, Hkv, G;
+  const uint16_t* q;
+  const uint16_t* k;
+  const uint16_t* v;
+  const int64_t* kv_off;
+  const int32_t* seq_len;
+  int max_T;
+  // gather (reuse) only
+  const int32_t* idx;
+  const int32_t* idx_k;
+  const int32_t* head_map;
+  int k_max;
+  float scale;
+  uint16_t* out;
+  float* lse;
+  float* pooled;  // anchor only
+  int64_t ld_pooled;
+  void* ws;
+  unsigned* status;
+};
+
+// Split geometry: each warp walks `tok_per_warp` items, 4 warps per CTA.
+struct DecodeSplit {
+  int tok_per_warp;
+  int nsplit;  // CTAs per (b, h)
+};
+DecodeSplit decode_split_for(int units, int n_items);
+size_t decode_workspace_bytes(int B, int Hkv, int G, int n_items, bool with_logits);
+
+cudaError_t launch_decode_anchor(const DecodeParams& p, cudaStream_t st);
+cudaError_t launch_decode_reuse(const DecodeParams& p, cudaStream_t st);
+
+// ------------------------------------------------------------------ topk ----
+size_t topk_smem_bytes(int64_t ld);
+cudaError_t launch_topk(const float* scores, int rows, int64_t ld, const int32_t* row_len,
+                        const int32_t* row_k, int k_max, int32_t* idx_out, unsigned* status,
+                        cudaStream_t st);
+
+// --------------------------------------------------------------- prefill ----
+struct PrefillParams {
+  int B, Hq, Hkv, G, N;
+  const uint16_t* q;
+  const uint16_t* k;
+  const uint16_t* v;
+  const int32_t* idx;
+  const int32_t* idx_k;
+  const int32_t* head_map;
+  int k_max;
+  float scale;
+  uint16_t* out;
+  float* lse;
+  float* pooled;
+  void* ws;
+  unsigned* status;
+};
+size_t prefill_anchor_workspace_bytes(int B, int Hq, int Hkv, int N);
+size_t prefill_reuse_workspace_bytes(int B, int Hq, int Hkv, int N, int k_max);
+cudaError_t launch_prefill_anchor(const PrefillParams& p, cudaStream_t st);
+cudaError_t launch_prefill_reuse(const PrefillParams& p, cudaStream_t st);
+
+}  // namespace kascade

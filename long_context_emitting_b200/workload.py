@@ -59,6 +59,7 @@ class DecodeConfig:
     anchors: Tuple[int, ...]
     heavy_frac: float
     T_range: Optional[Tuple[int, int]] = None
+    T_list: Optional[Tuple[int, ...]] = None   # explicit per-sequence lengths
     plant: float = 3.0
     drift: float = 0.0
     sink_tokens: int = 0
@@ -70,6 +71,8 @@ class DecodeConfig:
     model: str = "Llama-3.1-8B attention shape"
 
     def seq_lens(self) -> list:
+        if self.T_list is not None:
+            return [int(x) for x in self.T_list]
         if self.T is not None:
             return [int(self.T)] * self.B
         lo, hi = self.T_range
@@ -255,3 +258,33 @@ def random_scores(rows: int, n: int, seed: int, kind: str = "uniform") -> torch.
     if kind == "equal":
         return torch.full((rows, n), 0.25)
     raise ValueError(kind)
+
+
+def decode_sequence(cfg: DecodeConfig, layer: int, b: int, device="cpu") -> dict:
+    """Sequence b of :func:`decode_layer` alone (same seeds per role):
+    q bf16 [Hq, d], k / v bf16 [Hkv, T_b, d]."""
+    T = cfg.seq_lens()[b]
+    u = directions(cfg, layer, device)
+    k = torch.stack([_keys(cfg, u[b, h], b, h, T, layer, device) for h in range(cfg.Hkv)])
+    v = torch.stack([_values(cfg, b, h, T, layer, device) for h in range(cfg.Hkv)])
+    gq = _gen(device, cfg.name, "Q", layer)
+    G = cfg.Hq // cfg.Hkv
+    q = cfg.q_dir * u.repeat_interleave(G, dim=1) + torch.randn(
+        cfg.B, cfg.Hq, cfg.d, generator=gq, device=device)
+    return {"q": q[b].to(torch.bfloat16), "k": k.to(torch.bfloat16), "v": v.to(torch.bfloat16),
+            "T": T}
+
+
+def prefill_group(cfg: PrefillConfig, layer: int, b: int, h: int, device="cpu") -> dict:
+    """KV head h of :func:`prefill_layer` with its query heads alone:
+    q bf16 [G, N, d], k / v bf16 [N, d]."""
+    G = cfg.Hq // cfg.Hkv
+    u = directions(cfg, layer, device)
+    k = _keys(cfg, u[b, h], b, h, cfg.N, layer, device)
+    v = _values(cfg, b, h, cfg.N, layer, device)
+    qs = []
+    for g in range(h * G, (h + 1) * G):
+        gq = _gen(device, cfg.name, "Q", layer, b, g)
+        qs.append(cfg.q_dir * u[b, h] + torch.randn(cfg.N, cfg.d, generator=gq, device=device))
+    return {"q": torch.stack(qs).to(torch.bfloat16), "k": k.to(torch.bfloat16),
+            "v": v.to(torch.bfloat16)}
