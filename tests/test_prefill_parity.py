@@ -1,0 +1,124 @@
+"""Prefill path (causal anchor with tile pooling -> Top-k -> reuse with the
+diagonal block) against the float64 oracle, on whole small inputs and on
+sampled query tiles of the 16K and 64K workloads."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from long_context_emitting_b200 import api, workload
+from long_context_emitting_b200.schedule import PrefillSchedule
+from _compare import (assert_attention_close, assert_index_set_ok, assert_pooled_close,
+                      LSE_ABS)
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda")
+SCALE = api.default_scale()
+TILE = 128
+
+
+def _np(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def _rows(tiles):
+    return np.concatenate([np.arange(TILE * t, TILE * t + TILE) for t in tiles])
+
+
+def _check(cfg, tiles=None, reuse_layer=1, b=0):
+    N = cfg.N
+    nt = N // TILE
+    tiles = list(range(nt)) if tiles is None else tiles
+    sch = PrefillSchedule(cfg.B, cfg.Hq, cfg.Hkv, N, (0,), 2, DEV)
+    a_in = workload.prefill_layer(cfg, 0, DEV)
+    out_a = torch.empty_like(a_in["q"])
+    sch.run_anchor(a_in, out_a)
+    lse_a = sch.lse.clone()
+    sch.run_topk()
+    hm = workload.head_map(cfg, reuse_layer).to(DEV)
+    r_in = workload.prefill_layer(cfg, reuse_layer, DEV)
+    out_r = torch.empty_like(r_in["q"])
+    sch.run_reuse(r_in, hm, out_r)
+    assert api.device_status() == 0
+
+    q, k, v = (_np(a_in[n][b]) for n in ("q", "k", "v"))
+    o_ref, lse_ref, pooled_ref = O.prefill_anchor(q, k, v, SCALE, tile=TILE, tiles=tiles)
+    rows = _rows(tiles)
+    assert_attention_close(_np(out_a[b])[:, rows], o_ref[:, rows], "prefill anchor O")
+    np.testing.assert_allclose(_np(lse_a[b])[:, rows], lse_ref[:, rows], atol=LSE_ABS, rtol=0)
+    pooled_gpu = sch.pooled[b].cpu().numpy()
+    idx_gpu = sch.idx[b].cpu().numpy()
+    k_max = sch.k_max
+    idx_ref = np.full((nt, cfg.Hkv, k_max), -1, dtype=np.int64)
+    idx_k = np.zeros((nt, cfg.Hkv), dtype=np.int64)
+    for t in tiles:
+        P = TILE * t
+        kt = O.k_for_len(P)
+        idx_k[t] = kt
+        for h in range(cfg.Hkv):
+            assert_pooled_close(pooled_gpu[t, h, :P], pooled_ref[t, h, :P], f"pooled t={t} h={h}")
+            exact = O.topk_select(pooled_gpu[t, h, :P].astype(np.float32), kt)
+            assert np.array_equal(idx_gpu[t, h, :kt], exact), f"topk t={t} h={h}"
+            assert (idx_gpu[t, h, kt:] == -1).all()
+            ref = O.topk_select(pooled_ref[t, h, :P], kt)
+            idx_ref[t, h, :kt] = ref
+            assert_index_set_ok(idx_gpu[t, h], ref, pooled_ref[t, h, :P], kt, f"t={t} h={h}")
+
+    hm_np = hm.cpu().numpy()
+    qr, kr, vr = (_np(r_in[n][b]) for n in ("q", "k", "v"))
+    got = _np(out_r[b])[:, rows]
+    o_a, lse_ra = O.prefill_reuse(qr, kr, vr, idx_gpu.astype(np.int64), idx_k, hm_np, SCALE,
+                                  tile=TILE, tiles=tiles)
+    assert_attention_close(got, o_a[:, rows], "prefill reuse O (GPU indices)")
+    np.testing.assert_allclose(_np(sch.lse[b])[:, rows], lse_ra[:, rows], atol=LSE_ABS, rtol=0)
+    o_b, _ = O.prefill_reuse(qr, kr, vr, idx_ref, idx_k, hm_np, SCALE, tile=TILE, tiles=tiles)
+    assert_attention_close(got, o_b[:, rows], "prefill reuse O (oracle indices)")
+
+
+def test_prefill_small_all_tiles():
+    cfg = workload.scaled(workload.PREFILL_16K, name="prefill_small", N=640)
+    _check(cfg)
+
+
+def test_prefill_batch2():
+    cfg = workload.scaled(workload.PREFILL_16K, name="prefill_b2", N=384, B=2)
+    _check(cfg, b=1)
+
+
+def test_prefill_n16384_sampled_tiles():
+    _check(workload.PREFILL_16K, tiles=[0, 1, 10, 11, 64, 127])
+
+
+def test_prefill_n65536_sampled_tiles():
+    _check(workload.PREFILL_64K, tiles=[0, 2, 300, 511])
+
+
+def test_prefill_reuse_full_prefix_is_dense():
+    cfg = workload.scaled(workload.PREFILL_16K, name="prefill_dense_eq", N=512)
+    inp = workload.prefill_layer(cfg, 0, DEV)
+    out_a, lse_a, _ = api.prefill_anchor(inp["q"], inp["k"], inp["v"], SCALE)
+    nt = cfg.N // TILE
+    k_max = cfg.N - TILE
+    idx = torch.full((1, nt, cfg.Hkv, k_max), -1, dtype=torch.int32)
+    idx_k = torch.zeros(1, nt, cfg.Hkv, dtype=torch.int32)
+    for t in range(nt):
+        idx[0, t, :, : TILE * t] = torch.arange(TILE * t, dtype=torch.int32)
+        idx_k[0, t] = TILE * t
+    hm = torch.arange(cfg.Hkv, dtype=torch.int32).flip(0)
+    out_r, lse_r = api.prefill_reuse(inp["q"], inp["k"], inp["v"], idx.to(DEV),
+                                     idx_k.view(-1).to(DEV), hm.to(DEV), SCALE)
+    assert api.device_status() == 0
+    assert np.abs(_np(out_a) - _np(out_r)).max() <= 8e-3
+    np.testing.assert_allclose(_np(lse_a), _np(lse_r), atol=LSE_ABS)
+
+
+def test_prefill_reuse_bad_index_sets_status():
+    cfg = workload.scaled(workload.PREFILL_16K, name="prefill_bad", N=256)
+    inp = workload.prefill_layer(cfg, 0, DEV)
+    idx = torch.zeros(1, 2, cfg.Hkv, 128, dtype=torch.int32)
+    idx[0, 1, :, :] = torch.arange(128, dtype=torch.int32)
+    idx[0, 1, 2, 7] = 128  # not before the tile start
+    idx_k = torch.tensor([0] * cfg.Hkv + [128] * cfg.Hkv, dtype=torch.int32)
+    hm = torch.arange(cfg.Hkv, dtype=torch.int32)
+    api.prefill_reuse(inp["q"], inp["k"], inp["v"], idx.to(DEV), idx_k.to(DEV), hm.to(DEV), SCALE)
+    assert api.device_status() == 5

@@ -63,11 +63,12 @@ def test_topk_ragged_rows_and_short_rows():
 
 @pytest.mark.parametrize("n,rows", [(32768, 3), (49152, 2), (49153, 2), (65536, 2), (131072, 2)])
 def test_topk_long_rows_cached_and_streamed(n, rows):
-    # rows beyond 49152 keys are re-read from global memory on every pass
-    scores = workload.random_scores(rows, n, seed=5, kind="uniform")
-    _check(scores, [n] * rows, [O.k_for_len(n)] * rows)
-    ties = workload.random_scores(rows, n, seed=6, kind="ties")
-    _check(ties, [n] * rows, [O.k_for_len(n)] * rows)
+    # rows beyond 49152 keys are re-read from global memory on every pass;
+    # the row stride is padded to a multiple of 4 floats (16-byte rows)
+    ld = (n + 3) // 4 * 4
+    for seed, kind in ((5, "uniform"), (6, "ties")):
+        scores = workload.random_scores(rows, ld, seed=seed, kind=kind)
+        _check(scores, [n] * rows, [O.k_for_len(n)] * rows)
 
 
 def test_topk_pooled_like_rows():
