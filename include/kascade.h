@@ -88,6 +88,37 @@ int kascade_decode_anchor(kascade_shape s, const uint16_t* q, const uint16_t* k,
                           float* pooled, int64_t ld_pooled, void* ws, size_t ws_bytes,
                           void* stream);
 
+/* Size of the library-owned scratch array used by kascade_decode_anchor_static_ws. */
+#define KASCADE_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+/* Decode anchor without caller-provided scratch.  The paper has no counterpart of
+ * this entry point; it exists for callers that cannot allocate device memory at
+ * the point where they run the layer: an inference-runtime plugin whose enqueue
+ * step may not allocate, or a serving engine that has handed nearly all device
+ * memory to its KV-cache pool up front (and cudaMalloc / cudaFree would also
+ * synchronise the device in the middle of a step).
+ *
+ * Same arguments, results and checks as kascade_decode_anchor, minus ws/ws_bytes.
+ * The scratch is a file-scope device array of KASCADE_STATIC_SCRATCH_BYTES that
+ * every GPU which loads the library holds until the process exits.  The call
+ * allocates nothing (no cudaMalloc, cudaFree or allocating library routine).
+ *   - Problems whose scratch, kascade_decode_anchor_workspace_bytes(s, max_T), is
+ *     larger than KASCADE_STATIC_SCRATCH_BYTES are refused with
+ *     KASCADE_ERR_WORKSPACE_TOO_SMALL before anything is launched.
+ *   - The first call on a device looks up the array's device address with
+ *     cudaGetSymbolAddress (this may load the library's kernels on that device);
+ *     make that first call before any stream capture.
+ *   - Every call, from any stream or thread, shares the one array per device, and
+ *     the array keeps the previous call's contents.  Calls whose kernels overlap on
+ *     the GPU race on it and corrupt each other's results: order them (one stream,
+ *     or events).  No part of the array needs to start at zero, because each call
+ *     writes every scratch element it later reads. */
+int kascade_decode_anchor_static_ws(kascade_shape s, const uint16_t* q, const uint16_t* k,
+                                    const uint16_t* v, const int64_t* kv_off,
+                                    const int32_t* seq_len, int32_t max_T, float scale,
+                                    uint16_t* out, float* lse, float* pooled,
+                                    int64_t ld_pooled, void* stream);
+
 /* ------------------------------------------------------------------------- */
 /* Row-wise Top-k select.  [explainer] 技術的詳細 › アンカーレイヤーと再利用レイヤー (exact Top-k
  * indices in anchor layers) and › Top-k設定 (k).  Ties are broken toward the lower index;

@@ -13,6 +13,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libkascade.so")
 
 KASCADE_OK = 0
+STATIC_SCRATCH_BYTES = 16 * 1024 * 1024  # KASCADE_STATIC_SCRATCH_BYTES in include/kascade.h
 STATUS_NAMES = {
     0: "KASCADE_OK",
     1: "KASCADE_ERR_INVALID_ARG",
@@ -28,6 +29,7 @@ EXPORTS = (
     "kascade_k_for_len",
     "kascade_decode_anchor_workspace_bytes",
     "kascade_decode_anchor",
+    "kascade_decode_anchor_static_ws",
     "kascade_topk_workspace_bytes",
     "kascade_topk",
     "kascade_decode_reuse_workspace_bytes",
@@ -63,6 +65,8 @@ _SIGNATURES = {
     "kascade_decode_anchor_workspace_bytes": (_SZ, [Shape, _I32]),
     "kascade_decode_anchor": (ctypes.c_int, [Shape, _P, _P, _P, _P, _P, _I32, _F, _P, _P, _P, _I64,
                                              _P, _SZ, _P]),
+    "kascade_decode_anchor_static_ws": (ctypes.c_int, [Shape, _P, _P, _P, _P, _P, _I32, _F, _P, _P,
+                                                       _P, _I64, _P]),
     "kascade_topk_workspace_bytes": (_SZ, [_I32, _I64]),
     "kascade_topk": (ctypes.c_int, [_P, _I32, _I64, _P, _P, _I32, _P, _P, _SZ, _P]),
     "kascade_decode_reuse_workspace_bytes": (_SZ, [Shape, _I32]),

@@ -1,0 +1,60 @@
+// kascade_decode_anchor_static_ws: the decode anchor with its scratch memory in
+// a fixed array that the library itself owns, for callers that must not
+// allocate device memory while they run (see include/kascade.h).
+//
+// The array lives in this file as a file-scope __device__ object.  Host code
+// cannot use its name as a device address, so the address is looked up once
+// per device with cudaGetSymbolAddress and handed to the regular launcher.
+#include "../../include/kascade.h"
+#include "internal.h"
+
+#include <cuda_runtime.h>
+
+namespace kascade {
+
+static __device__ __align__(256) unsigned char g_static_scratch[KASCADE_STATIC_SCRATCH_BYTES];
+
+}  // namespace kascade
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+// Device address of g_static_scratch on the current device, looked up on the
+// first call per device (the lookup may load the module on that device, which
+// is why the first call should not happen inside a stream capture).
+void* static_scratch_address() {
+  static void* cache[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  if (!cache[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, kascade::g_static_scratch) != cudaSuccess) return nullptr;
+    cache[dev] = p;
+  }
+  return cache[dev];
+}
+
+}  // namespace
+
+extern "C" int kascade_decode_anchor_static_ws(kascade_shape s, const uint16_t* q,
+                                               const uint16_t* k, const uint16_t* v,
+                                               const int64_t* kv_off, const int32_t* seq_len,
+                                               int32_t max_T, float scale, uint16_t* out,
+                                               float* lse, float* pooled, int64_t ld_pooled,
+                                               void* stream) {
+  // Size check first, so an oversized request is refused without touching CUDA.
+  const size_t need = kascade_decode_anchor_workspace_bytes(s, max_T);
+  if (need > (size_t)KASCADE_STATIC_SCRATCH_BYTES) return KASCADE_ERR_WORKSPACE_TOO_SMALL;
+  // A bad shape (size 0) or an empty batch launches nothing: let the regular
+  // entry point report it without looking up the scratch array.
+  if (need == 0 || s.B == 0)
+    return kascade_decode_anchor(s, q, k, v, kv_off, seq_len, max_T, scale, out, lse, pooled,
+                                 ld_pooled, nullptr, 0, stream);
+  void* ws = static_scratch_address();
+  if (!ws) return KASCADE_ERR_CUDA;
+  // Nothing in the scratch needs to start at zero: every partial and logit the
+  // combine step reads is written earlier in the same call.
+  return kascade_decode_anchor(s, q, k, v, kv_off, seq_len, max_T, scale, out, lse, pooled,
+                               ld_pooled, ws, (size_t)KASCADE_STATIC_SCRATCH_BYTES, stream);
+}
