@@ -78,11 +78,8 @@ class Dist:
             self.pg.barrier()
 
     def max(self, x: float) -> float:
-        if not self.pg:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
-        return float(t.item())
+        from long_context_emitting_b200 import replicas
+        return replicas.max_over_ranks(x, self.pg, "cuda")
 
     def close(self):
         if self.pg:
@@ -135,11 +132,11 @@ class Clocks:
 
 
 # --------------------------------------------------------------------------------------
-def build_decode(dev, n_layers=None):
-    from long_context_emitting_b200 import workload
+def build_decode(dev, n_layers=None, rank=0):
+    from long_context_emitting_b200 import replicas, workload
     from long_context_emitting_b200.schedule import DecodeSchedule
 
-    cfg = workload.DECODE_32K
+    cfg = replicas.rank_workload(workload.DECODE_32K, rank)
     L = cfg.n_layers if n_layers is None else n_layers
     lens = cfg.seq_lens()
     sch = DecodeSchedule(cfg.B, cfg.Hq, cfg.Hkv, lens, cfg.anchors, L, dev)
@@ -149,11 +146,11 @@ def build_decode(dev, n_layers=None):
     return cfg, sch, layers, maps, outs
 
 
-def build_prefill(dev):
-    from long_context_emitting_b200 import workload
+def build_prefill(dev, rank=0):
+    from long_context_emitting_b200 import replicas, workload
     from long_context_emitting_b200.schedule import PrefillSchedule
 
-    cfg = workload.PREFILL_16K
+    cfg = replicas.rank_workload(workload.PREFILL_16K, rank)
     sch = PrefillSchedule(cfg.B, cfg.Hq, cfg.Hkv, cfg.N, cfg.anchors, cfg.n_layers, dev)
     layers = [workload.prefill_layer(cfg, l, dev) for l in range(cfg.n_layers)]
     maps = {l: workload.head_map(cfg, l).to(dev) for l in range(cfg.n_layers) if l not in cfg.anchors}
@@ -349,8 +346,8 @@ def main():
     do_dec = args.only in ("all", "decode")
     do_pre = args.only in ("all", "prefill")
 
-    dec = build_decode(dev, args.decode_layers) if do_dec else None
-    pre = build_prefill(dev) if do_pre else None
+    dec = build_decode(dev, args.decode_layers, dist.rank) if do_dec else None
+    pre = build_prefill(dev, dist.rank) if do_pre else None
     torch.cuda.synchronize()
 
     def step(timer=None):
@@ -397,7 +394,8 @@ def main():
         n_anchor = sum(1 for l in range(L) if sch.is_anchor(l))
         dec_ms = dist.max((timer.total_ms("dec_anchor") + timer.total_ms("dec_topk")
                            + timer.total_ms("dec_reuse")) / args.steps)
-        us_layer = dec_ms * 1e3 / (L * N)
+        from long_context_emitting_b200.replicas import whole_job_us_per_layer
+        us_layer = whole_job_us_per_layer(dec_ms, L, N)
         anchor_ms = timer.mean_ms("dec_anchor")
         topk_ms = timer.mean_ms("dec_topk")
         reuse_ms = timer.mean_ms("dec_reuse")

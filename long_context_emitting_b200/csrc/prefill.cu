@@ -1,28 +1,39 @@
 // Prefill-phase Kascade kernels on the 5th-generation tensor cores
-// (tcgen05.mma, accumulators in tensor memory, operands in 128-byte-swizzled
-// shared memory filled by TMA or cp.async).
+// (tcgen05.mma with accumulators in tensor memory, operands in 128-byte-
+// swizzled shared memory filled by TMA).
 //
 // Method: Kascade explainer (0h-n0.github.io), 主要な貢献 (tile-level
 // post-softmax pooling in prefill), 実装のポイント (128-query tiles),
 // 技術的詳細 › アンカーレイヤーと再利用レイヤー and › ヘッドリマッピング.
 //
-// prefill_attn_kernel<GATHER>: one CTA (128 threads, thread r <-> query row r
-//   <-> TMEM lane r) per (query tile t, query head g, sequence b).
-//   * anchor (GATHER = false): key blocks 0..t of the causal row, loaded by TMA;
-//     block t is the diagonal block and is masked causally.
-//   * reuse (GATHER = true): the anchor's indices of row (t, head_map[h]) in
-//     blocks of 128 gathered rows (cp.async into the same swizzled layout),
-//     then the diagonal block.
-//   Per block: S = Q K^T into TMEM (8 MMAs of K = 16), each thread reads its
-//   row, online softmax in base 2 (the running maximum is only raised when a
-//   block exceeds it by more than 2^8, so the O accumulator in TMEM is rarely
-//   rescaled), P (bf16) goes to shared memory, O += P V into TMEM.
-//   Epilogue: O / l to bf16 and the natural-log LSE.
-// prefill_pool_kernel: one CTA per (tile t >= 1, KV head h, sequence b).  For
-//   each key block before the tile it computes S^T = K Q_g^T for the group's
-//   query heads (keys on TMEM lanes, queries on columns), so each thread owns
-//   one key and sums exp2(s - lse2) over the 128 queries x G heads in
-//   registers; pooled = sum / (128 G).
+// prefill_attn_kernel<GATHER>
+//   One CTA per (query tile t, pair of query heads of one GQA group, sequence).
+//   The two heads share every K/V block, so each block is loaded once for two
+//   128 x 128 attention tiles.  Warp roles (384 threads):
+//     warp 0      TMA producer: Q tiles, then K/V blocks into a 2-stage ring.
+//                 anchor: dense key blocks 0..t (block t is the diagonal);
+//                 reuse: the anchor's indices of row (t, head_map[h]) gathered
+//                 with cp.async (two whole rows per warp instruction) into the
+//                 same swizzled layout, then the diagonal block by TMA.
+//     warp 1      MMA issuer (one thread): S_i = Q_i K^T into TMEM, and
+//                 O_i += P_i V with P_i read from TMEM (it overwrites S_i).
+//     warps 4-7   softmax of tile 0, warps 8-11 softmax of tile 1: thread r
+//                 owns query row r (TMEM lane r), reads S, runs the online
+//                 softmax in base 2 (the running maximum is raised only when a
+//                 block exceeds it by 2^8, so O is rarely rescaled), writes P
+//                 back to TMEM as bf16 and finally normalises O.
+//   The MMA thread alternates between the tiles, so the tensor cores work on
+//   one tile while the other tile's softmax runs.
+//   TMEM (512 columns): S0|P0 [0,128), O0 [128,256), S1|P1 [256,384), O1 [384,512).
+//
+// prefill_pool_kernel
+//   One CTA per (tile t >= 1, KV head, sequence).  For each key block before
+//   the tile it computes S^T = K Q_g^T for the group's query heads (keys on
+//   TMEM lanes, queries on columns), so a thread owns one key and sums
+//   exp2(s - lse2) over the tile's queries in registers.  Warp roles: a TMA
+//   producer, an MMA issuer and two warpgroups that each sum half of the heads
+//   (ping-ponging on two TMEM regions); the two halves are added through shared
+//   memory and pooled = sum / (128 G) is written once, without atomics.
 #include "tcgen05.cuh"
 #include "internal.h"
 
@@ -35,27 +46,31 @@ namespace kascade {
 namespace {
 
 constexpr int kTile = 128;
-constexpr int kThreads = 128;
 constexpr uint32_t kHalfBytes = 128u * 128u;     // 64 bf16 columns x 128 rows (one TMA box)
 constexpr uint32_t kTileBytes = 2u * kHalfBytes;  // 128 x 128 bf16
 constexpr float kRescaleLog2 = 8.f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2e = 1.4426950408889634f;
 
-// shared-memory map of the attention kernel (offsets from a 1024-aligned base)
-constexpr uint32_t kAttnQ = 0;
-constexpr uint32_t kAttnK = kTileBytes;                 // 2 stages
-constexpr uint32_t kAttnV = kAttnK + 2 * kTileBytes;    // 2 stages
-constexpr uint32_t kAttnP = kAttnV + 2 * kTileBytes;
-constexpr uint32_t kAttnMisc = kAttnP + kTileBytes;
-constexpr uint32_t kAttnSmem = kAttnMisc + 2048 + 1024;  // misc + alignment slack
+// ---- attention kernel layout ----
+constexpr int kAttnThreads = 384;
+constexpr uint32_t kAttnQ = 0;                         // 2 query tiles
+constexpr uint32_t kAttnKV = 2 * kTileBytes;           // stage s: K at +2s*tile, V at +(2s+1)*tile
+constexpr uint32_t kAttnMisc = kAttnKV + 4 * kTileBytes;
+constexpr uint32_t kAttnSmem = kAttnMisc + 256 + 1024;  // misc + alignment slack
+enum { kBarQ = 0, kBarKvFull = 1, kBarKvEmpty = 3, kBarS = 5, kBarP = 7, kBarO = 9, kAttnBars = 11 };
 
-// shared-memory map of the pooling kernel
+// ---- pooling kernel layout ----
+constexpr int kPoolThreads = 384;
 constexpr int kPoolHeads = 4;                           // query heads resident at once
-constexpr uint32_t kPoolQ = 0;                          // kPoolHeads tiles
+constexpr uint32_t kPoolQ = 0;
 constexpr uint32_t kPoolK = kPoolHeads * kTileBytes;    // 2 stages
-constexpr uint32_t kPoolMisc = kPoolK + 2 * kTileBytes;
-constexpr uint32_t kPoolSmem = kPoolMisc + kPoolHeads * kTile * 4 + 1024 + 1024;
+constexpr uint32_t kPoolLse = kPoolK + 2 * kTileBytes;  // [kPoolHeads][128] floats
+constexpr uint32_t kPoolRed = kPoolLse + kPoolHeads * kTile * 4;  // [2][128] floats
+constexpr uint32_t kPoolMisc = kPoolRed + 2 * kTile * 4;
+constexpr uint32_t kPoolSmem = kPoolMisc + 256 + 1024;
+enum { kPBarQ = 0, kPBarKFull = 1, kPBarKEmpty = 3, kPBarS = 5, kPBarFree = 7, kPBarRedFull = 9,
+       kPBarRedEmpty = 11, kPoolBars = 13 };
 
 struct AttnArgs {
   int B, Hq, Hkv, G, N, n_tiles;
@@ -79,11 +94,6 @@ struct PoolArgs {
   unsigned* status;
 };
 
-__device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t chunk16) {
-  // byte offset of 16-byte chunk `chunk16` (0..15) of row `row` in a 128 x 128 bf16 tile
-  return (chunk16 >> 3) * kHalfBytes + row * 128u + (((chunk16 & 7u) ^ (row & 7u)) << 4);
-}
-
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int ks) {
   return sw128_desc(tile + (uint32_t)(ks >> 2) * kHalfBytes + (uint32_t)(ks & 3) * 32u, 16u, 1024u);
 }
@@ -91,27 +101,31 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile, int ks) {
   return sw128_desc(tile + (uint32_t)ks * 2048u, kHalfBytes, 1024u);
 }
 
+__device__ __forceinline__ volatile int* abort_flag(uint8_t* smem, uint32_t misc) {
+  return reinterpret_cast<volatile int*>(smem + misc + 128);
+}
+
 template <bool GATHER>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kAttnThreads, 1)
 prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kAttnMisc);   // q, kv0, kv1, s, o
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kAttnMisc + 64);
-  int* s_abort = reinterpret_cast<int*>(smem + kAttnMisc + 68);
-  uint8_t* valid = smem + kAttnMisc + 128;                          // [2][128] (gather)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kAttnMisc);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kAttnMisc + 96);
+  volatile int* s_abort = abort_flag(smem, kAttnMisc);
+  uint32_t* masks = reinterpret_cast<uint32_t*>(smem + kAttnMisc + 160);  // [2 stages][4]
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int t = a.n_tiles - 1 - (int)blockIdx.x;  // longest rows first
-  const int g = blockIdx.y, b = blockIdx.z;
-  const int h = g / a.G;
-  const uint32_t bar_q = smem_u32(&bars[0]);
-  const uint32_t bar_s = smem_u32(&bars[3]);
-  const uint32_t bar_o = smem_u32(&bars[4]);
+  const int b = blockIdx.z;
+  const int ntile = a.G >= 2 ? 2 : 1;
+  const int g0 = blockIdx.y * ntile;
+  const int h = g0 / a.G;
 
-  // ---- which key blocks ------------------------------------------------------
+  // ---- key blocks ------------------------------------------------------------
   int n_gather = 0, kt = 0;
   const int32_t* irow = nullptr;
   if (GATHER) {
@@ -130,238 +144,15 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     n_gather = (kt + kTile - 1) / kTile;
   }
   const int nblk = GATHER ? n_gather + 1 : t + 1;
-  const int64_t q_row0 = ((int64_t)b * a.Hq + g) * a.N + (int64_t)kTile * t;
-  const int64_t kv_row0 = ((int64_t)b * a.Hkv + h) * a.N;
+  const int64_t q_row0 = ((int64_t)b * a.Hq + g0) * a.N + (int64_t)kTile * t;
+  const int kv_row0 = (int)(((int64_t)b * a.Hkv + h) * a.N);
 
   if (tid == 0) {
-    for (int i = 0; i < 5; ++i) mbar_init(smem_u32(&bars[i]), 1);
+    for (int i = 0; i < kAttnBars; ++i) mbar_init(bar(i), (i == kBarP || i == kBarP + 1) ? 128u : 1u);
     *s_abort = 0;
     mbar_fence_init();
   }
-  if (warp == 0) {
-    tmem_alloc(smem_u32(tmem_slot), 256);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tO = tmem + 128;
-  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-
-  auto load_block = [&](int jb, int stage) {
-    const uint32_t ks = sbase + kAttnK + stage * kTileBytes;
-    const uint32_t vs = sbase + kAttnV + stage * kTileBytes;
-    if (!GATHER) {
-      if (tid == 0) {
-        const uint32_t bar = smem_u32(&bars[1 + stage]);
-        mbar_expect_tx(bar, 2 * kTileBytes);
-        const int y = (int)(kv_row0 + (int64_t)kTile * jb);
-        tma_load_2d(ks, &tm_k, 0, y, bar);
-        tma_load_2d(ks + kHalfBytes, &tm_k, 64, y, bar);
-        tma_load_2d(vs, &tm_v, 0, y, bar);
-        tma_load_2d(vs + kHalfBytes, &tm_v, 64, y, bar);
-      }
-    } else {
-      const bool diag = jb == n_gather;
-      for (int e = tid; e < kTile * 16; e += kThreads) {
-        const int row = e >> 4, c16 = e & 15;
-        int key;
-        bool ok;
-        if (diag) {
-          key = kTile * t + row;
-          ok = true;
-        } else {
-          const int pos = kTile * jb + row;
-          key = pos < kt ? __ldg(irow + pos) : -1;
-          ok = key >= 0 && key < kTile * t;
-          if (pos < kt && !ok && c16 == 0) flag_status(a.status, kStatusBadIndex);
-        }
-        const int64_t src_row = kv_row0 + (ok ? key : 0);
-        const uint32_t off = swz(row, c16);
-        cp_async16(ks + off, a.k + src_row * kHeadDim + c16 * 8, ok ? 16u : 0u);
-        cp_async16(vs + off, a.v + src_row * kHeadDim + c16 * 8, ok ? 16u : 0u);
-        if (c16 == 0) valid[stage * kTile + row] = ok ? 1 : 0;
-      }
-      cp_async_commit();
-    }
-  };
-
-  if (tid == 0) {
-    mbar_expect_tx(bar_q, kTileBytes);
-    tma_load_2d(sbase + kAttnQ, &tm_q, 0, (int)q_row0, bar_q);
-    tma_load_2d(sbase + kAttnQ + kHalfBytes, &tm_q, 64, (int)q_row0, bar_q);
-  }
-  load_block(0, 0);
-
-  const uint32_t idesc_s = idesc_bf16(128, 128, false, false);
-  const uint32_t idesc_o = idesc_bf16(128, 128, false, true);
-  const int r = tid;
-  float m_used = -INFINITY, l_sum = 0.f;
-  bool failed = false;
-
-  for (int it = 0; it < nblk; ++it) {
-    const int stage = it & 1;
-    if (it + 1 < nblk) load_block(it + 1, stage ^ 1);
-    if (GATHER) {
-      if (it + 1 < nblk) cp_async_wait<1>(); else cp_async_wait<0>();
-      fence_proxy_async_smem();
-      __syncthreads();
-    }
-    // ---- S = Q K^T --------------------------------------------------------
-    if (tid == 0) {
-      bool ok = true;
-      if (it == 0) ok = mbar_wait(bar_q, 0, a.status);
-      if (!GATHER && ok) ok = mbar_wait(smem_u32(&bars[1 + stage]), (it >> 1) & 1, a.status);
-      if (ok) {
-        tc_fence_after();
-        const uint32_t qs = sbase + kAttnQ, ksm = sbase + kAttnK + stage * kTileBytes;
-#pragma unroll
-        for (int k16 = 0; k16 < 8; ++k16)
-          umma_ss(tS, kmajor_desc(qs, k16), kmajor_desc(ksm, k16), idesc_s, k16 > 0 ? 1u : 0u);
-        umma_commit(bar_s);
-      } else {
-        *s_abort = 1;
-      }
-    }
-    __syncthreads();
-    if (*s_abort) { failed = true; break; }
-    if (!mbar_wait(bar_s, it & 1, a.status)) { *s_abort = 1; }
-    tc_fence_after();
-
-    // ---- softmax on row r ---------------------------------------------------
-    uint32_t sr[4][32];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) tmem_ld32(tS + lane_base + 32 * c, sr[c]);
-    tmem_wait_ld();
-    const bool is_diag = GATHER ? (it == n_gather) : (it == t);
-    const uint8_t* vflags = valid + stage * kTile;
-    float mloc = -INFINITY;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-#pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const int col = 32 * c + e;
-        bool ok = is_diag ? (col <= r) : (!GATHER || vflags[col]);
-        float x = ok ? __uint_as_float(sr[c][e]) * a.scale_log2 : -INFINITY;
-        sr[c][e] = __float_as_uint(x);
-        mloc = fmaxf(mloc, x);
-      }
-    }
-    float alpha = 1.f;
-    bool rescale = false;
-    if (m_used == -INFINITY) {
-      m_used = mloc;
-    } else if (mloc > m_used + kRescaleLog2) {
-      alpha = fast_exp2(m_used - mloc);
-      m_used = mloc;
-      rescale = true;
-    }
-    const float base = (m_used == -INFINITY) ? 0.f : m_used;
-    l_sum *= alpha;
-    uint8_t* prow = smem + kAttnP;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-#pragma unroll
-      for (int q8 = 0; q8 < 4; ++q8) {  // 8 keys -> one 16-byte chunk
-        uint32_t w[4];
-#pragma unroll
-        for (int e2 = 0; e2 < 4; ++e2) {
-          const float p0 = fast_exp2(__uint_as_float(sr[c][8 * q8 + 2 * e2]) - base);
-          const float p1 = fast_exp2(__uint_as_float(sr[c][8 * q8 + 2 * e2 + 1]) - base);
-          l_sum += p0 + p1;
-          w[e2] = pack_bf16x2(p0, p1);
-        }
-        const uint32_t chunk = (uint32_t)(4 * c + q8);  // keys 8*chunk .. 8*chunk+7
-        *reinterpret_cast<uint4*>(prow + swz((uint32_t)r, chunk)) = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-    }
-    if (__any_sync(0xffffffffu, rescale) && it > 0) {
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t o[32];
-        tmem_ld32(tO + lane_base + 32 * c, o);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-        tmem_st32(tO + lane_base + 32 * c, o);
-      }
-      tmem_wait_st();
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    // ---- O += P V ---------------------------------------------------------
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t ps = sbase + kAttnP, vsm = sbase + kAttnV + stage * kTileBytes;
-#pragma unroll
-      for (int k16 = 0; k16 < 8; ++k16)
-        umma_ss(tO, kmajor_desc(ps, k16), mnmajor_desc(vsm, k16), idesc_o,
-                (it > 0 || k16 > 0) ? 1u : 0u);
-      umma_commit(bar_o);
-    }
-    if (!mbar_wait(bar_o, it & 1, a.status)) { *s_abort = 1; }
-    tc_fence_after();
-    __syncthreads();
-    if (*s_abort) { failed = true; break; }
-  }
-
-  // ---- epilogue ---------------------------------------------------------------
-  if (!failed) {
-    const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
-    uint16_t* orow = a.out + (q_row0 + r) * kHeadDim;
-#pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-      uint32_t o[32];
-      tmem_ld32(tO + lane_base + 32 * c, o);
-      tmem_wait_ld();
-#pragma unroll
-      for (int q8 = 0; q8 < 4; ++q8) {
-        uint4 w;
-        w.x = pack_bf16x2(__uint_as_float(o[8 * q8 + 0]) * inv_l, __uint_as_float(o[8 * q8 + 1]) * inv_l);
-        w.y = pack_bf16x2(__uint_as_float(o[8 * q8 + 2]) * inv_l, __uint_as_float(o[8 * q8 + 3]) * inv_l);
-        w.z = pack_bf16x2(__uint_as_float(o[8 * q8 + 4]) * inv_l, __uint_as_float(o[8 * q8 + 5]) * inv_l);
-        w.w = pack_bf16x2(__uint_as_float(o[8 * q8 + 6]) * inv_l, __uint_as_float(o[8 * q8 + 7]) * inv_l);
-        *reinterpret_cast<uint4*>(orow + 32 * c + 8 * q8) = w;
-      }
-    }
-    if (a.lse) a.lse[q_row0 + r] = l_sum > 0.f ? (m_used + __log2f(l_sum)) * kLn2 : -INFINITY;
-  }
-  if (GATHER) cp_async_wait<0>();
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 256);
-  }
-}
-
-__global__ void __launch_bounds__(kThreads, 1)
-prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const PoolArgs a) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const uint32_t sbase = smem_u32(smem);
-  float* lse2 = reinterpret_cast<float*>(smem + kPoolMisc);                   // [kPoolHeads][128]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kPoolMisc + kPoolHeads * kTile * 4);  // q, k0, k1, s
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
-  int* s_abort = reinterpret_cast<int*>(bars + 9);
-
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int t = a.n_tiles - 1 - (int)blockIdx.x;  // t >= 1, longest first
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int G = a.G;
-  const uint32_t bar_q = smem_u32(&bars[0]);
-  const uint32_t bar_s = smem_u32(&bars[3]);
-  const int64_t kv_row0 = ((int64_t)b * a.Hkv + h) * a.N;
-
-  if (tid == 0) {
-    for (int i = 0; i < 4; ++i) mbar_init(smem_u32(&bars[i]), 1);
-    *s_abort = 0;
-    mbar_fence_init();
-  }
-  if (warp == 0) {
+  if (warp == 2) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
@@ -369,95 +160,373 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-  const uint32_t idesc = idesc_bf16(128, 128, false, false);
-  float* prow = a.pooled + (((int64_t)b * a.n_tiles + t) * a.Hkv + h) * a.N;
-  const float inv_count = 1.f / (float)(kTile * G);
 
-  int it = 0;        // global block counter (K stage / phase bookkeeping)
-  int q_phase = 0;
-  bool failed = false;
-  for (int g0 = 0; g0 < G && !failed; g0 += kPoolHeads) {
-    const int hg = min(kPoolHeads, G - g0);
-    // queries of the heads in this round, and their log2-domain LSE
-    if (tid == 0) {
-      mbar_expect_tx(bar_q, hg * kTileBytes);
-      for (int j = 0; j < hg; ++j) {
-        const int y = (int)(((int64_t)b * a.Hq + h * G + g0 + j) * a.N + (int64_t)kTile * t);
-        tma_load_2d(sbase + kPoolQ + j * kTileBytes, &tm_q, 0, y, bar_q);
-        tma_load_2d(sbase + kPoolQ + j * kTileBytes + kHalfBytes, &tm_q, 64, y, bar_q);
+  if (warp == 0) {
+    // ================================ TMA producer ================================
+    if (lane == 0) {
+      mbar_expect_tx(bar(kBarQ), ntile * kTileBytes);
+      for (int i = 0; i < ntile; ++i) {
+        const int y = (int)(q_row0 + (int64_t)i * a.N);
+        tma_load_2d(sbase + kAttnQ + i * kTileBytes, &tm_q, 0, y, bar(kBarQ));
+        tma_load_2d(sbase + kAttnQ + i * kTileBytes + kHalfBytes, &tm_q, 64, y, bar(kBarQ));
       }
     }
-    for (int e = tid; e < hg * kTile; e += kThreads) {
-      const int j = e / kTile, i = e % kTile;
-      lse2[e] = a.lse[((int64_t)b * a.Hq + h * G + g0 + j) * a.N + (int64_t)kTile * t + i] * kLog2e;
-    }
-    auto load_k = [&](int jb, int stage) {
-      if (tid == 0) {
-        const uint32_t bar = smem_u32(&bars[1 + stage]);
-        mbar_expect_tx(bar, kTileBytes);
-        const int y = (int)(kv_row0 + (int64_t)kTile * jb);
-        const uint32_t ks = sbase + kPoolK + stage * kTileBytes;
-        tma_load_2d(ks, &tm_k, 0, y, bar);
-        tma_load_2d(ks + kHalfBytes, &tm_k, 64, y, bar);
-      }
-    };
-    load_k(0, it & 1);
-    __syncthreads();  // lse2 visible
-    for (int jb = 0; jb < t; ++jb, ++it) {
-      const int stage = it & 1;
-      if (jb + 1 < t) load_k(jb + 1, stage ^ 1);
-      if (tid == 0) {
-        bool ok = true;
-        if (jb == 0) ok = mbar_wait(bar_q, q_phase, a.status);
-        if (ok) ok = mbar_wait(smem_u32(&bars[1 + stage]), (it >> 1) & 1, a.status);
-        if (ok) {
-          tc_fence_after();
-          const uint32_t ks = sbase + kPoolK + stage * kTileBytes;
-          for (int j = 0; j < hg; ++j) {
-            const uint32_t qs = sbase + kPoolQ + j * kTileBytes;
+    for (int j = 0; j < nblk; ++j) {
+      const int st = j & 1;
+      if (j >= 2 && !mbar_wait(bar(kBarKvEmpty + st), ((j >> 1) - 1) & 1, a.status)) { *s_abort = 1; break; }
+      if (*s_abort) break;
+      const uint32_t kb = sbase + kAttnKV + (2 * st) * kTileBytes;
+      const uint32_t vb = kb + kTileBytes;
+      const bool dense = !GATHER || j == n_gather;
+      if (dense) {
+        if (lane == 0) {
+          mbar_expect_tx(bar(kBarKvFull + st), 2 * kTileBytes);
+          const int y = kv_row0 + kTile * (GATHER ? t : j);
+          tma_load_2d(kb, &tm_k, 0, y, bar(kBarKvFull + st));
+          tma_load_2d(kb + kHalfBytes, &tm_k, 64, y, bar(kBarKvFull + st));
+          tma_load_2d(vb, &tm_v, 0, y, bar(kBarKvFull + st));
+          tma_load_2d(vb + kHalfBytes, &tm_v, 64, y, bar(kBarKvFull + st));
+        }
+      } else {
+        // Gathered block: validity of rows 4*lane .. 4*lane+3 -> 4 ballot words.
+        uint32_t m[4];
 #pragma unroll
-            for (int k16 = 0; k16 < 8; ++k16)
-              umma_ss(tmem + 128 * j, kmajor_desc(ks, k16), kmajor_desc(qs, k16), idesc,
-                      k16 > 0 ? 1u : 0u);
-          }
-          umma_commit(bar_s);
-        } else {
-          *s_abort = 1;
+        for (int e = 0; e < 4; ++e) {
+          const int pos = kTile * j + 4 * lane + e;
+          const int key = pos < kt ? __ldg(irow + pos) : -1;
+          const bool ok = key >= 0 && key < kTile * t;
+          if (pos < kt && !ok) flag_status(a.status, kStatusBadIndex);
+          m[e] = __ballot_sync(0xffffffffu, ok);
+        }
+        // Copy: each warp instruction moves two whole 256-byte rows (16 lanes per
+        // row, one 16-byte chunk each) into the swizzled layout; masked rows are
+        // zero-filled from a valid address.
+        const int c16 = lane & 15;
+        const uint32_t half = (uint32_t)(c16 >> 3) * kHalfBytes;
+        for (int s2 = 0; s2 < kTile / 2; ++s2) {
+          const int row = 2 * s2 + (lane >> 4);
+          const int pos = kTile * j + row;
+          const int key = pos < kt ? __ldg(irow + pos) : -1;
+          const bool ok = key >= 0 && key < kTile * t;
+          const int64_t src = (int64_t)kv_row0 + (ok ? key : kTile * t);
+          const uint32_t off = half + (uint32_t)row * 128u + ((uint32_t)((c16 & 7) ^ (row & 7)) << 4);
+          cp_async16(kb + off, a.k + src * kHeadDim + c16 * 8, ok ? 16u : 0u);
+          cp_async16(vb + off, a.v + src * kHeadDim + c16 * 8, ok ? 16u : 0u);
+        }
+        cp_async_commit();
+        cp_async_wait<0>();
+        fence_proxy_async_smem();  // the tensor cores read these rows through the async proxy
+        __syncwarp();
+        if (lane == 0) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) masks[st * 4 + e] = m[e];
+          mbar_arrive(bar(kBarKvFull + st));  // release: rows and masks visible
         }
       }
-      __syncthreads();
-      if (*s_abort) { failed = true; break; }
-      if (!mbar_wait(bar_s, it & 1, a.status)) { failed = true; }
-      tc_fence_after();
-      float acc = 0.f;
-      for (int j = 0; j < hg; ++j) {
-        const float* l2 = lse2 + j * kTile;
+    }
+  } else if (warp == 1) {
+    // ================================ MMA issuer ==================================
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16(128, 128, false, false);
+      const uint32_t idesc_o = idesc_bf16(128, 128, false, true);
+      auto issue_s = [&](int i, uint32_t kb) {
+        const uint32_t qs = sbase + kAttnQ + i * kTileBytes;
+#pragma unroll
+        for (int k16 = 0; k16 < 8; ++k16)
+          umma_ss(tmem + 256 * i, kmajor_desc(qs, k16), kmajor_desc(kb, k16), idesc_s, k16 > 0 ? 1u : 0u);
+      };
+      auto issue_pv = [&](int i, uint32_t vb, bool acc) {
+#pragma unroll
+        for (int k16 = 0; k16 < 8; ++k16)
+          umma_ts(tmem + 256 * i + 128, tmem + 256 * i + 8 * k16, mnmajor_desc(vb, k16), idesc_o,
+                  (acc || k16 > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(bar(kBarQ), 0, a.status);
+      for (int j = 0; ok && j < nblk; ++j) {
+        const int st = j & 1;
+        const uint32_t kb = sbase + kAttnKV + (2 * st) * kTileBytes;
+        const uint32_t vb = kb + kTileBytes;
+        if (!(ok = mbar_wait(bar(kBarKvFull + st), (j >> 1) & 1, a.status))) break;
+        tc_fence_after();
+        if (j == 0) {
+          for (int i = 0; i < ntile; ++i) {
+            issue_s(i, kb);
+            umma_commit(bar(kBarS + i));
+          }
+        }
+        const bool more = j + 1 < nblk;
+        const uint32_t kb2 = sbase + kAttnKV + (2 * (st ^ 1)) * kTileBytes;
+        // tile 0: PV of this block, then S of the next block
+        if (!(ok = mbar_wait(bar(kBarP + 0), j & 1, a.status))) break;
+        tc_fence_after();
+        issue_pv(0, vb, j > 0);
+        if (more) {
+          if (!(ok = mbar_wait(bar(kBarKvFull + (st ^ 1)), ((j + 1) >> 1) & 1, a.status))) break;
+          tc_fence_after();
+          issue_s(0, kb2);
+          umma_commit(bar(kBarS + 0));
+        }
+        if (ntile == 2) {
+          if (!(ok = mbar_wait(bar(kBarP + 1), j & 1, a.status))) break;
+          tc_fence_after();
+          issue_pv(1, vb, j > 0);
+        }
+        umma_commit(bar(kBarKvEmpty + st));  // K/V stage free once these MMAs complete
+        if (ntile == 2 && more) {
+          issue_s(1, kb2);
+          umma_commit(bar(kBarS + 1));
+        }
+        if (*s_abort) { ok = false; break; }
+      }
+      if (!ok) *s_abort = 1;
+      for (int i = 0; i < ntile; ++i) umma_commit(bar(kBarO + i));
+    }
+  } else if (warp >= 4) {
+    // ================================ softmax =====================================
+    const int i = (warp - 4) >> 2;  // tile
+    const int r = tid - 128 - 128 * i;  // query row = TMEM lane
+    if (i < ntile) {
+      const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+      const uint32_t tS = tmem + 256 * i + lane_base;
+      const uint32_t tO = tS + 128;
+      float m_used = -INFINITY, l_sum = 0.f;
+      bool ok = true;
+      for (int j = 0; j < nblk; ++j) {
+        if (!(ok = mbar_wait(bar(kBarS + i), j & 1, a.status)) || *s_abort) { ok = false; break; }
+        tc_fence_after();
+        const bool diag = GATHER ? (j == n_gather) : (j == t);
+        uint32_t mk[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
+        if (GATHER && !diag) {
+          if (!(ok = mbar_wait(bar(kBarKvFull + (j & 1)), (j >> 1) & 1, a.status))) break;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) mk[e] = masks[(j & 1) * 4 + e];
+        }
+        uint32_t sr[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
+        tmem_wait_ld();
+        float mloc = -INFINITY;
+#pragma unroll
+        for (int col = 0; col < 128; ++col) {
+          bool keep = diag ? (col <= r) : (((mk[col & 3] >> (col >> 2)) & 1u) != 0u);
+          const float x = keep ? __uint_as_float(sr[col]) * a.scale_log2 : -INFINITY;
+          sr[col] = __float_as_uint(x);
+          mloc = fmaxf(mloc, x);
+        }
+        float alpha = 1.f;
+        bool rescale = false;
+        if (m_used == -INFINITY) {
+          m_used = mloc;
+        } else if (mloc > m_used + kRescaleLog2) {
+          alpha = fast_exp2(m_used - mloc);
+          m_used = mloc;
+          rescale = true;
+        }
+        if (__any_sync(0xffffffffu, rescale) && j > 0) {
+          // the previous PV of this tile completed before S of this block was committed
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + 32 * c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(tO + 32 * c, o);
+          }
+        }
+        l_sum *= alpha;
+        const float base = (m_used == -INFINITY) ? 0.f : m_used;
+        uint32_t pw[64];
+#pragma unroll
+        for (int c2 = 0; c2 < 64; ++c2) {
+          const float p0 = fast_exp2(__uint_as_float(sr[2 * c2]) - base);
+          const float p1 = fast_exp2(__uint_as_float(sr[2 * c2 + 1]) - base);
+          l_sum += p0 + p1;
+          pw[c2] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pw[0]));
+        tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pw[32]));
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(kBarP + i));
+      }
+      if (!ok) *s_abort = 1;
+      // ---- epilogue: O / l ----------------------------------------------------
+      if (mbar_wait(bar(kBarO + i), 0, a.status) && ok && !*s_abort) {
+        tc_fence_after();
+        const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
+        const int64_t orow_i = q_row0 + (int64_t)i * a.N + r;
+        uint16_t* orow = a.out + orow_i * kHeadDim;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
-          uint32_t sv[32];
-          tmem_ld32(tmem + 128 * j + lane_base + 32 * c, sv);
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * c, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            acc += fast_exp2(__uint_as_float(sv[e]) * a.scale_log2 - l2[32 * c + e]);
+          for (int q8 = 0; q8 < 4; ++q8) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(o[8 * q8 + 0]) * inv_l, __uint_as_float(o[8 * q8 + 1]) * inv_l);
+            w.y = pack_bf16x2(__uint_as_float(o[8 * q8 + 2]) * inv_l, __uint_as_float(o[8 * q8 + 3]) * inv_l);
+            w.z = pack_bf16x2(__uint_as_float(o[8 * q8 + 4]) * inv_l, __uint_as_float(o[8 * q8 + 5]) * inv_l);
+            w.w = pack_bf16x2(__uint_as_float(o[8 * q8 + 6]) * inv_l, __uint_as_float(o[8 * q8 + 7]) * inv_l);
+            *reinterpret_cast<uint4*>(orow + 32 * c + 8 * q8) = w;
+          }
         }
+        if (a.lse) a.lse[orow_i] = l_sum > 0.f ? (m_used + __log2f(l_sum)) * kLn2 : -INFINITY;
       }
-      const int key = kTile * jb + tid;
-      if (g0 == 0) prow[key] = acc * inv_count;
-      else prow[key] += acc * inv_count;
-      tc_fence_before();
-      __syncthreads();
-      if (failed) *s_abort = 1;
-      __syncthreads();
-      if (*s_abort) { failed = true; break; }
     }
-    q_phase ^= 1;
-    __syncthreads();  // Q tiles and lse2 are replaced by the next round
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+__global__ void __launch_bounds__(kPoolThreads, 1)
+prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const PoolArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  float* lse2 = reinterpret_cast<float*>(smem + kPoolLse);
+  float* red = reinterpret_cast<float*>(smem + kPoolRed);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kPoolMisc);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kPoolMisc + 96);
+  volatile int* s_abort = abort_flag(smem, kPoolMisc);
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int t = a.n_tiles - 1 - (int)blockIdx.x;  // t >= 1, longest first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int G = a.G;
+  const int kv_row0 = (int)(((int64_t)b * a.Hkv + h) * a.N);
+  const int n_rounds = (G + kPoolHeads - 1) / kPoolHeads;
+  const int nblk = t;  // key blocks before the tile, per round
+
+  if (tid == 0) {
+    for (int i = 0; i < kPoolBars; ++i)
+      mbar_init(bar(i), i >= kPBarFree ? 128u : 1u);
+    *s_abort = 0;
+    mbar_fence_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  float* prow = a.pooled + (((int64_t)b * a.n_tiles + t) * a.Hkv + h) * a.N;
+  const float inv_count = 1.f / (float)(kTile * G);
+
+  for (int rd = 0; rd < n_rounds; ++rd) {
+    const int hg = min(kPoolHeads, G - rd * kPoolHeads);  // heads this round
+    const int gbase = h * G + rd * kPoolHeads;
+    // lse of the round's heads (log2 domain), read by the summing warps
+    for (int e = tid; e < hg * kTile; e += kPoolThreads) {
+      const int j = e / kTile, q = e % kTile;
+      lse2[e] = a.lse[((int64_t)b * a.Hq + gbase + j) * a.N + (int64_t)kTile * t + q] * kLog2e;
+    }
+    __syncthreads();
+    const int it0 = rd * nblk;  // running block counter for stage / phase bookkeeping
+    if (warp == 0) {
+      // ---------------------------- TMA producer ----------------------------
+      if (lane == 0) {
+        mbar_expect_tx(bar(kPBarQ), hg * kTileBytes);
+        for (int j = 0; j < hg; ++j) {
+          const int y = (int)(((int64_t)b * a.Hq + gbase + j) * a.N + (int64_t)kTile * t);
+          tma_load_2d(sbase + kPoolQ + j * kTileBytes, &tm_q, 0, y, bar(kPBarQ));
+          tma_load_2d(sbase + kPoolQ + j * kTileBytes + kHalfBytes, &tm_q, 64, y, bar(kPBarQ));
+        }
+        for (int jb = 0; jb < nblk; ++jb) {
+          const int it = it0 + jb, st = it & 1;
+          if (it >= 2 && !mbar_wait(bar(kPBarKEmpty + st), ((it >> 1) - 1) & 1, a.status)) { *s_abort = 1; break; }
+          if (*s_abort) break;
+          const uint32_t ks = sbase + kPoolK + st * kTileBytes;
+          mbar_expect_tx(bar(kPBarKFull + st), kTileBytes);
+          tma_load_2d(ks, &tm_k, 0, kv_row0 + kTile * jb, bar(kPBarKFull + st));
+          tma_load_2d(ks + kHalfBytes, &tm_k, 64, kv_row0 + kTile * jb, bar(kPBarKFull + st));
+        }
+      }
+    } else if (warp == 1) {
+      // ---------------------------- MMA issuer ------------------------------
+      if (lane == 0) {
+        const uint32_t idesc = idesc_bf16(128, 128, false, false);
+        bool ok = mbar_wait(bar(kPBarQ), rd & 1, a.status);
+        for (int jb = 0; ok && jb < nblk; ++jb) {
+          const int it = it0 + jb, st = it & 1;
+          if (!(ok = mbar_wait(bar(kPBarKFull + st), (it >> 1) & 1, a.status))) break;
+          const uint32_t ks = sbase + kPoolK + st * kTileBytes;
+          for (int w = 0; w < 2; ++w) {
+            // region w holds heads 2w, 2w+1 of the round; wait until its summing
+            // warpgroup has read the previous block
+            if (it >= 1 && !(ok = mbar_wait(bar(kPBarFree + w), (it - 1) & 1, a.status))) break;
+            tc_fence_after();
+            for (int jj = 2 * w; jj < min(2 * w + 2, hg); ++jj) {
+              const uint32_t qs = sbase + kPoolQ + jj * kTileBytes;
+#pragma unroll
+              for (int k16 = 0; k16 < 8; ++k16)
+                umma_ss(tmem + 128 * jj, kmajor_desc(ks, k16), kmajor_desc(qs, k16), idesc,
+                        k16 > 0 ? 1u : 0u);
+            }
+            umma_commit(bar(kPBarS + w));
+          }
+          if (!ok) break;
+          umma_commit(bar(kPBarKEmpty + st));
+          if (*s_abort) { ok = false; break; }
+        }
+        if (!ok) *s_abort = 1;
+      }
+    } else if (warp >= 4) {
+      // ------------------- summing warpgroups (heads 2w, 2w+1) ---------------
+      const int w = (warp - 4) >> 2;
+      const int key = tid - 128 - 128 * w;  // TMEM lane
+      const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+      for (int jb = 0; jb < nblk; ++jb) {
+        const int it = it0 + jb;
+        if (!mbar_wait(bar(kPBarS + w), it & 1, a.status) || *s_abort) { *s_abort = 1; break; }
+        tc_fence_after();
+        float acc = 0.f;
+        for (int jj = 2 * w; jj < min(2 * w + 2, hg); ++jj) {
+          const float* l2 = lse2 + jj * kTile;
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t sv[32];
+            tmem_ld32(tmem + 128 * jj + lane_base + 32 * c, sv);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              acc += fast_exp2(__uint_as_float(sv[e]) * a.scale_log2 - l2[32 * c + e]);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bar(kPBarFree + w));
+        // add the two warpgroups' halves (exchange slot double-buffered by block
+        // parity, guarded by bounded mbarrier waits) and write the pooled value
+        const int sl = it & 1;
+        float* slot = red + sl * kTile;
+        if (w == 1) {
+          if (it >= 2 && !mbar_wait(bar(kPBarRedEmpty + sl), ((it >> 1) - 1) & 1, a.status)) { *s_abort = 1; break; }
+          slot[key] = acc;
+          mbar_arrive(bar(kPBarRedFull + sl));
+        } else {
+          if (!mbar_wait(bar(kPBarRedFull + sl), (it >> 1) & 1, a.status)) { *s_abort = 1; break; }
+          const float tot = acc + slot[key];
+          mbar_arrive(bar(kPBarRedEmpty + sl));
+          const int col = kTile * jb + key;
+          if (rd == 0) prow[col] = tot * inv_count;
+          else prow[col] += tot * inv_count;
+        }
+      }
+    }
+    __syncthreads();  // round done: Q tiles and lse2 may be replaced
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -476,13 +545,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D view [rows, 128] bf16, box of 64 columns x 128 rows, 128-byte swizzle.
-bool make_tile_map(CUtensorMap* map, const void* base, uint64_t rows) {
+// 2-D view [rows, 128] bf16, boxes of 64 columns x box_rows rows, 128-byte swizzle.
+bool make_tile_map(CUtensorMap* map, const void* base, uint64_t rows, uint32_t box_rows) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * 2};
-  cuuint32_t box[2] = {64, 128};
+  cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -497,28 +566,29 @@ size_t prefill_reuse_workspace_bytes(int, int, int, int, int) { return 0; }
 
 static cudaError_t launch_attn(const PrefillParams& p, bool gather, cudaStream_t st) {
   const int n_tiles = p.N / kTile;
+  const uint64_t kv_rows = (uint64_t)p.B * p.Hkv * p.N;
+  if (kv_rows >= (1ull << 31) || (uint64_t)p.B * p.Hq * p.N >= (1ull << 31)) return cudaErrorNotSupported;
   CUtensorMap tq, tk, tv;
-  if (!make_tile_map(&tq, p.q, (uint64_t)p.B * p.Hq * p.N) ||
-      !make_tile_map(&tk, p.k, (uint64_t)p.B * p.Hkv * p.N) ||
-      !make_tile_map(&tv, p.v, (uint64_t)p.B * p.Hkv * p.N))
+  if (!make_tile_map(&tq, p.q, (uint64_t)p.B * p.Hq * p.N, 128) || !make_tile_map(&tk, p.k, kv_rows, 128) ||
+      !make_tile_map(&tv, p.v, kv_rows, 128))
     return cudaErrorInvalidValue;
   AttnArgs a;
   a.B = p.B; a.Hq = p.Hq; a.Hkv = p.Hkv; a.G = p.G; a.N = p.N; a.n_tiles = n_tiles;
-  a.k = p.k; a.v = p.v; a.idx = p.idx; a.idx_k = p.idx_k; a.head_map = p.head_map;
-  a.k_max = p.k_max;
+  a.k = p.k; a.v = p.v;
+  a.idx = p.idx; a.idx_k = p.idx_k; a.head_map = p.head_map; a.k_max = p.k_max;
   a.scale_log2 = (float)((double)p.scale * 1.4426950408889634);
   a.out = p.out; a.lse = p.lse; a.status = p.status;
-  dim3 grid(n_tiles, p.Hq, p.B);
+  const int ntile = p.G >= 2 ? 2 : 1;
+  dim3 grid(n_tiles, p.Hq / ntile, p.B);
+  cudaError_t e;
   if (gather) {
-    cudaError_t e = cudaFuncSetAttribute(prefill_attn_kernel<true>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem);
+    e = cudaFuncSetAttribute(prefill_attn_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem);
     if (e != cudaSuccess) return e;
-    prefill_attn_kernel<true><<<grid, kThreads, kAttnSmem, st>>>(tq, tk, tv, a);
+    prefill_attn_kernel<true><<<grid, kAttnThreads, kAttnSmem, st>>>(tq, tk, tv, a);
   } else {
-    cudaError_t e = cudaFuncSetAttribute(prefill_attn_kernel<false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem);
+    e = cudaFuncSetAttribute(prefill_attn_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem);
     if (e != cudaSuccess) return e;
-    prefill_attn_kernel<false><<<grid, kThreads, kAttnSmem, st>>>(tq, tk, tv, a);
+    prefill_attn_kernel<false><<<grid, kAttnThreads, kAttnSmem, st>>>(tq, tk, tv, a);
   }
   return cudaGetLastError();
 }
@@ -529,8 +599,8 @@ cudaError_t launch_prefill_anchor(const PrefillParams& p, cudaStream_t st) {
   const int n_tiles = p.N / kTile;
   if (n_tiles < 2) return cudaSuccess;
   CUtensorMap tq, tk;
-  if (!make_tile_map(&tq, p.q, (uint64_t)p.B * p.Hq * p.N) ||
-      !make_tile_map(&tk, p.k, (uint64_t)p.B * p.Hkv * p.N))
+  if (!make_tile_map(&tq, p.q, (uint64_t)p.B * p.Hq * p.N, 128) ||
+      !make_tile_map(&tk, p.k, (uint64_t)p.B * p.Hkv * p.N, 128))
     return cudaErrorInvalidValue;
   PoolArgs a;
   a.B = p.B; a.Hq = p.Hq; a.Hkv = p.Hkv; a.G = p.G; a.N = p.N; a.n_tiles = n_tiles;
@@ -539,7 +609,7 @@ cudaError_t launch_prefill_anchor(const PrefillParams& p, cudaStream_t st) {
   e = cudaFuncSetAttribute(prefill_pool_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPoolSmem);
   if (e != cudaSuccess) return e;
   dim3 grid(n_tiles - 1, p.Hkv, p.B);
-  prefill_pool_kernel<<<grid, kThreads, kPoolSmem, st>>>(tq, tk, a);
+  prefill_pool_kernel<<<grid, kPoolThreads, kPoolSmem, st>>>(tq, tk, a);
   return cudaGetLastError();
 }
 
