@@ -158,6 +158,66 @@ def build_prefill(dev, rank=0):
     return cfg, sch, layers, maps, outs
 
 
+class _Cudart:
+    """The CUDA runtime torch already loaded, for event-record nodes inside graphs."""
+
+    def __init__(self):
+        import ctypes
+        self.ct = ctypes
+        self.lib = ctypes.CDLL("libcudart.so.12")
+        self.lib.cudaEventCreate.argtypes = [ctypes.POINTER(ctypes.c_void_p)]
+        self.lib.cudaEventRecordWithFlags.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint]
+        self.lib.cudaEventElapsedTime.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.c_void_p,
+                                                  ctypes.c_void_p]
+        self.lib.cudaEventDestroy.argtypes = [ctypes.c_void_p]
+
+    def create(self):
+        ev = self.ct.c_void_p()
+        assert self.lib.cudaEventCreate(self.ct.byref(ev)) == 0
+        return ev
+
+    def record_external(self, ev):
+        # cudaEventRecordExternal = 1: a real event-record node when captured
+        rc = self.lib.cudaEventRecordWithFlags(ev, self.ct.c_void_p(torch.cuda.current_stream().cuda_stream), 1)
+        assert rc == 0, rc
+
+    def elapsed_ms(self, a, b) -> float:
+        ms = self.ct.c_float()
+        assert self.lib.cudaEventElapsedTime(self.ct.byref(ms), a, b) == 0
+        return ms.value
+
+
+class GraphOpTimer:
+    """Event-record nodes around every op of a captured step.  After each
+    replay, ``collect()`` adds the per-op device times of that replay."""
+
+    def __init__(self, rt: _Cudart):
+        self.rt = rt
+        self.marks = []       # (name, start_event, end_event) in capture order
+        self.times = {}
+
+    def run(self, name, fn, *args):
+        s, e = self.rt.create(), self.rt.create()
+        self.rt.record_external(s)
+        fn(*args)
+        self.rt.record_external(e)
+        self.marks.append((name, s, e))
+
+    def collect(self):
+        for name, s, e in self.marks:
+            self.times.setdefault(name, []).append(self.rt.elapsed_ms(s, e))
+
+    def span_ms(self):
+        return self.rt.elapsed_ms(self.marks[0][1], self.marks[-1][2])
+
+    def mean_ms(self, name):
+        v = self.times.get(name, [])
+        return sum(v) / len(v) if v else 0.0
+
+    def total_ms(self, name):
+        return sum(self.times.get(name, []))
+
+
 class OpTimer:
     """CUDA events around each call on the launching (current) stream."""
 
@@ -362,24 +422,45 @@ def main():
     if api.device_status() != 0:
         raise RuntimeError("device status set during warm-up")
 
+    # Each schedule step (all layers) is captured once as a CUDA graph, with
+    # event-record nodes around every op; the timed region replays the graphs.
+    from long_context_emitting_b200.schedule import StepGraph
+
+    rt = _Cudart()
+    timer = GraphOpTimer(rt)
+    capturing = torch.cuda.is_current_stream_capturing
+    gdec = StepGraph(lambda: decode_step(dec[1], dec[2], dec[3], dec[4],
+                                         timer if capturing() else None)) if dec else None
+    dec_marks = len(timer.marks)
+    gpre = StepGraph(lambda: prefill_step(pre[1], pre[2], pre[3], pre[4],
+                                          timer if capturing() else None)) if pre else None
+    if api.device_status() != 0:
+        raise RuntimeError("device status set during capture")
+
     clocks = Clocks(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
                     else int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[dist.local]))
-    timer = OpTimer()
     dist.barrier()
     torch.cuda.synchronize()
     clocks.start()
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    t_start.record()
+    step_ms, dec_ms_steps, pre_ms_steps = [], [], []
     for _ in range(args.steps):
-        step(timer)
-    t_end.record()
+        if gdec:
+            gdec.replay()
+        if gpre:
+            gpre.replay()
+        torch.cuda.synchronize()
+        timer.collect()
+        d = rt.elapsed_ms(timer.marks[0][1], timer.marks[dec_marks - 1][2]) if gdec else 0.0
+        p = rt.elapsed_ms(timer.marks[dec_marks][1], timer.marks[-1][2]) if gpre else 0.0
+        dec_ms_steps.append(d)
+        pre_ms_steps.append(p)
+        step_ms.append(d + p)
     torch.cuda.synchronize()
     dist.barrier()
     clk = clocks.stop()
-    timer.collect()
-    total_ms = dist.max(t_start.elapsed_time(t_end))
-    ms_per_step = total_ms / args.steps
+    if api.device_status() != 0:
+        raise RuntimeError("device status set during the timed steps")
+    ms_per_step = dist.max(sum(step_ms) / args.steps)
     N = dist.world
 
     out = {"metric": METRIC, "unit": UNIT, "n_gpus": N, "steps": args.steps,
@@ -392,8 +473,7 @@ def main():
         cfg, sch = dec[0], dec[1]
         L = sch.n_layers
         n_anchor = sum(1 for l in range(L) if sch.is_anchor(l))
-        dec_ms = dist.max((timer.total_ms("dec_anchor") + timer.total_ms("dec_topk")
-                           + timer.total_ms("dec_reuse")) / args.steps)
+        dec_ms = dist.max(sum(dec_ms_steps) / args.steps)
         from long_context_emitting_b200.replicas import whole_job_us_per_layer
         us_layer = whole_job_us_per_layer(dec_ms, L, N)
         anchor_ms = timer.mean_ms("dec_anchor")
@@ -427,8 +507,7 @@ def main():
                           "Hkv": cfg.Hkv, "d": cfg.d}
     if pre:
         cfg, sch = pre[0], pre[1]
-        pre_ms = dist.max((timer.total_ms("pre_anchor") + timer.total_ms("pre_topk")
-                           + timer.total_ms("pre_reuse")) / args.steps)
+        pre_ms = dist.max(sum(pre_ms_steps) / args.steps)
         pa = timer.mean_ms("pre_anchor")
         pt = timer.mean_ms("pre_topk")
         pr = timer.mean_ms("pre_reuse")
@@ -475,7 +554,8 @@ def main():
 def e2e(dec, pre, args, dist):
     """Same metric through the public API with pinned host buffers: every step
     copies its new queries (decode; the KV cache is device-resident state) or
-    its q/k/v (prefill) host->device and reads the outputs back."""
+    its q/k/v (prefill) host->device and reads the outputs back.  Copies and
+    kernels of a step are captured together in one CUDA graph."""
     h2d = d2h = 0
     res = {"unit": UNIT}
     if dec:
@@ -494,14 +574,13 @@ def e2e(dec, pre, args, dist):
             for l in range(L):
                 o_host[l].copy_(outs[l], non_blocking=True)
 
-        for _ in range(2):
-            dstep()
-        torch.cuda.synchronize()
+        from long_context_emitting_b200.schedule import StepGraph
+        g = StepGraph(dstep, warmup=2)
         dist.barrier()
         s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s.record()
         for _ in range(args.steps):
-            dstep()
+            g.replay()
         e.record()
         torch.cuda.synchronize()
         ms = dist.max(s.elapsed_time(e)) / args.steps
@@ -523,13 +602,13 @@ def e2e(dec, pre, args, dist):
             for l in range(L):
                 ho[l].copy_(outs[l], non_blocking=True)
 
-        pstep()
-        torch.cuda.synchronize()
+        from long_context_emitting_b200.schedule import StepGraph
+        g = StepGraph(pstep, warmup=1)
         dist.barrier()
         s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s.record()
         for _ in range(args.steps):
-            pstep()
+            g.replay()
         e.record()
         torch.cuda.synchronize()
         pms = dist.max(s.elapsed_time(e)) / args.steps

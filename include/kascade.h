@@ -149,7 +149,8 @@ int kascade_topk(const float* scores, int32_t rows, int64_t ld, const int32_t* r
  *   idx_k    int32 [B·Hkv]           valid count per anchor row, <= k_max
  *   head_map int32 [Hkv]             values in [0, Hkv)
  *   out bf16 [B, Hq, d]; lse fp32 [B, Hq] (may be NULL)
- *   ws       scratch of kascade_decode_reuse_workspace_bytes(s, k_max) bytes
+ *   ws       scratch of kascade_decode_reuse_workspace_bytes(s, k_max) bytes (currently 0:
+ *            the splits of a row merge on chip; NULL is accepted when the size is 0)
  * Out-of-range indices are skipped (status KASCADE_ERR_BAD_INDEX). */
 size_t kascade_decode_reuse_workspace_bytes(kascade_shape s, int32_t k_max);
 int kascade_decode_reuse(kascade_shape s, const uint16_t* q, const uint16_t* k,

@@ -125,13 +125,14 @@ int kascade_decode_reuse(kascade_shape s, const uint16_t* q, const uint16_t* k,
   if (rc) return rc;
   if (k_max < 0 || !std::isfinite(scale)) return KASCADE_ERR_INVALID_ARG;
   if (s.B == 0) return KASCADE_OK;
-  if (!q || !k || !v || !kv_off || !seq_len || !idx || !idx_k || !head_map || !out || !ws)
+  const size_t need = kascade_decode_reuse_workspace_bytes(s, k_max);
+  if (!q || !k || !v || !kv_off || !seq_len || !idx || !idx_k || !head_map || !out || (need && !ws))
     return KASCADE_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(ws) ||
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || (ws && !aligned16(ws)) ||
       (lse && !aligned16(lse)) || ((uintptr_t)kv_off & 7) || ((uintptr_t)seq_len & 3) ||
       ((uintptr_t)idx & 3) || ((uintptr_t)idx_k & 3) || ((uintptr_t)head_map & 3))
     return KASCADE_ERR_INVALID_ARG;
-  if (ws_bytes < kascade_decode_reuse_workspace_bytes(s, k_max)) return KASCADE_ERR_WORKSPACE_TOO_SMALL;
+  if (ws_bytes < need) return KASCADE_ERR_WORKSPACE_TOO_SMALL;
   DecodeParams p = {};
   p.B = s.B; p.Hq = s.Hq; p.Hkv = s.Hkv; p.G = s.Hq / s.Hkv;
   p.q = q; p.k = k; p.v = v; p.kv_off = kv_off; p.seq_len = seq_len;

@@ -25,6 +25,9 @@
 // into pooled probabilities, mean over the group's query heads.
 #include "common.cuh"
 #include "internal.h"
+#include "tcgen05.cuh"
+
+#include <cooperative_groups.h>
 
 #include <cmath>
 
@@ -55,6 +58,8 @@ struct SplitArgs {
   float* logits;   // anchor: [B, Hkv, max_T, G] base-2 scaled logits
   float* part_ml;  // [B*Hkv, nsplit, G, 2]  (running max, running sum)
   float* part_o;   // [B*Hkv, nsplit, G, 128] unnormalised output
+  uint16_t* out;      // reuse: written by rank 0 of each (b, h) cluster
+  float* lse;
   unsigned* status;
 };
 
@@ -86,8 +91,125 @@ __device__ __forceinline__ int resolve_rows(const SplitArgs& a, int b, int h, in
   return ok ? n : -1;
 }
 
+// One block of 16 items (tokens or gathered indices) held in registers.
+struct Blk {
+  uint4 ka[4], kb[4], va[4], vb[4];
+  int ia, ib;        // item positions (for the logits store)
+  bool oka, okb;     // rows present
+};
+
 template <bool GATHER>
-__global__ void __launch_bounds__(kThreads) decode_split_kernel(const SplitArgs a) {
+__device__ __forceinline__ void load_blk(Blk& x, int i0, int i_end, const int32_t* rows, int T,
+                                         const uint16_t* Kb, const uint16_t* Vb, int gid, int tig,
+                                         unsigned* status) {
+  x.ia = i0 + gid;
+  x.ib = i0 + gid + 8;
+  x.oka = x.ia < i_end;
+  x.okb = x.ib < i_end;
+  int ra = x.ia, rb = x.ib;
+  if (GATHER) {
+    ra = x.oka ? __ldg(rows + x.ia) : 0;
+    rb = x.okb ? __ldg(rows + x.ib) : 0;
+    if (x.oka && (ra < 0 || ra >= T)) { flag_status(status, kStatusBadIndex); x.oka = false; }
+    if (x.okb && (rb < 0 || rb >= T)) { flag_status(status, kStatusBadIndex); x.okb = false; }
+    // masked lanes address row 0 (T >= 1 here), so no address leaves the sequence
+    if (!x.oka) ra = 0;
+    if (!x.okb) rb = 0;
+  } else {
+    // masked lanes address the block's first row, which is < i_end <= T
+    if (!x.oka) ra = i0;
+    if (!x.okb) rb = i0;
+  }
+  const uint16_t* kpa = Kb + (int64_t)ra * kHeadDim + 8 * tig;
+  const uint16_t* kpb = Kb + (int64_t)rb * kHeadDim + 8 * tig;
+  const uint16_t* vpa = Vb + (int64_t)ra * kHeadDim + 8 * tig;
+  const uint16_t* vpb = Vb + (int64_t)rb * kHeadDim + 8 * tig;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    x.ka[j] = ldg_stream16(kpa + 32 * j);
+    x.kb[j] = ldg_stream16(kpb + 32 * j);
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    x.va[j] = ldg_stream16(vpa + 32 * j);
+    x.vb[j] = ldg_stream16(vpb + 32 * j);
+  }
+}
+
+struct WarpState {
+  float m0, m1, l0, l1;
+  float o[8][4];
+};
+
+template <bool GATHER>
+__device__ __forceinline__ void compute_blk(const Blk& x, WarpState& w, const uint32_t (&qf)[4][4],
+                                            float scale_log2, float* lrow, int G, int tig) {
+  // S^T = K · Q^T  (rows: items ia / ib; cols: heads 2tig, 2tig+1)
+  float s[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};  // two independent chains
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    mma_bf16_16816(s, word_of(x.ka[j], 0), word_of(x.kb[j], 0), word_of(x.ka[j], 1),
+                   word_of(x.kb[j], 1), qf[j][0], qf[j][1]);
+    mma_bf16_16816(s2, word_of(x.ka[j], 2), word_of(x.kb[j], 2), word_of(x.ka[j], 3),
+                   word_of(x.kb[j], 3), qf[j][2], qf[j][3]);
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) s[e] += s2[e];
+  s[0] = x.oka ? s[0] * scale_log2 : -INFINITY;
+  s[1] = x.oka ? s[1] * scale_log2 : -INFINITY;
+  s[2] = x.okb ? s[2] * scale_log2 : -INFINITY;
+  s[3] = x.okb ? s[3] * scale_log2 : -INFINITY;
+
+  if (!GATHER) {
+    if (2 * tig + 1 < G) {
+      if (x.oka) *reinterpret_cast<float2*>(lrow + (int64_t)x.ia * G + 2 * tig) = make_float2(s[0], s[1]);
+      if (x.okb) *reinterpret_cast<float2*>(lrow + (int64_t)x.ib * G + 2 * tig) = make_float2(s[2], s[3]);
+    } else if (2 * tig < G) {
+      if (x.oka) lrow[(int64_t)x.ia * G + 2 * tig] = s[0];
+      if (x.okb) lrow[(int64_t)x.ib * G + 2 * tig] = s[2];
+    }
+  }
+
+  // online softmax (base 2)
+  const float mx0 = warp_max_xor_gid(fmaxf(s[0], s[2]));
+  const float mx1 = warp_max_xor_gid(fmaxf(s[1], s[3]));
+  const float mn0 = fmaxf(w.m0, mx0), mn1 = fmaxf(w.m1, mx1);
+  const float base0 = (mn0 == -INFINITY) ? 0.f : mn0;
+  const float base1 = (mn1 == -INFINITY) ? 0.f : mn1;
+  const float al0 = fast_exp2(w.m0 - base0), al1 = fast_exp2(w.m1 - base1);
+  const float p0 = fast_exp2(s[0] - base0), p1 = fast_exp2(s[1] - base1);
+  const float p2 = fast_exp2(s[2] - base0), p3 = fast_exp2(s[3] - base1);
+  w.l0 = w.l0 * al0 + p0 + p2;
+  w.l1 = w.l1 * al1 + p1 + p3;
+  w.m0 = mn0;
+  w.m1 = mn1;
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) {
+    w.o[mt][0] *= al0; w.o[mt][1] *= al1; w.o[mt][2] *= al0; w.o[mt][3] *= al1;
+  }
+
+  // O^T += V^T · P^T
+  const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p0, p1));
+  const uint32_t pb1 = movmatrix_trans(pack_bf16x2(p2, p3));
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+#pragma unroll
+    for (int pp = 0; pp < 2; ++pp) {
+      const uint32_t a0 = movmatrix_trans(word_of(x.va[j], 2 * pp));
+      const uint32_t a1 = movmatrix_trans(word_of(x.va[j], 2 * pp + 1));
+      const uint32_t a2 = movmatrix_trans(word_of(x.vb[j], 2 * pp));
+      const uint32_t a3 = movmatrix_trans(word_of(x.vb[j], 2 * pp + 1));
+      mma_bf16_16816(w.o[2 * j + pp], a0, a1, a2, a3, pb0, pb1);
+    }
+  }
+}
+
+// Anchor (contiguous stream): two register buffers, the next block's loads in
+// flight during the current block's math, 2 CTAs per SM.  Reuse (gather): one
+// buffer and 4 CTAs per SM, since more resident warps hide the scattered-row
+// latency better than deeper per-warp pipelining.
+template <bool GATHER>
+__global__ void __launch_bounds__(kThreads, GATHER ? 4 : 2) decode_split_kernel(const SplitArgs a) {
   __shared__ float sm_o[kWarps][8][kHeadDim];
   __shared__ float sm_m[kWarps][8];
   __shared__ float sm_l[kWarps][8];
@@ -122,112 +244,42 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(const SplitArgs 
     qf[j][0] = t.x; qf[j][1] = t.y; qf[j][2] = t.z; qf[j][3] = t.w;
   }
 
-  float m_run0 = -INFINITY, m_run1 = -INFINITY;
-  float l_run0 = 0.f, l_run1 = 0.f;
-  float o[8][4];
+  WarpState ws;
+  ws.m0 = ws.m1 = -INFINITY;
+  ws.l0 = ws.l1 = 0.f;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  for (int i = 0; i < 8; ++i) ws.o[i][0] = ws.o[i][1] = ws.o[i][2] = ws.o[i][3] = 0.f;
 
   float* lrow = nullptr;
   if (!GATHER) lrow = a.logits + ((int64_t)b * a.Hkv + h) * a.max_T * G;
 
+  // Two register buffers: the next block's loads are in flight while the
+  // current block is computed.
+  if (!GATHER) {
+  Blk x0, x1;
+  if (i_begin < i_end) load_blk<GATHER>(x0, i_begin, i_end, rows, T, Kb, Vb, gid, tig, a.status);
+  for (int i0 = i_begin; i0 < i_end; i0 += 32) {
+    const bool has1 = i0 + 16 < i_end;
+    if (has1) load_blk<GATHER>(x1, i0 + 16, i_end, rows, T, Kb, Vb, gid, tig, a.status);
+    compute_blk<GATHER>(x0, ws, qf, a.scale_log2, lrow, G, tig);
+    if (!has1) break;
+    if (i0 + 32 < i_end) load_blk<GATHER>(x0, i0 + 32, i_end, rows, T, Kb, Vb, gid, tig, a.status);
+    compute_blk<GATHER>(x1, ws, qf, a.scale_log2, lrow, G, tig);
+  }
+  } else {
   for (int i0 = i_begin; i0 < i_end; i0 += 16) {
-    const int ia = i0 + gid, ib = i0 + gid + 8;
-    bool va = ia < i_end, vb = ib < i_end;
-    int ra = ia, rb = ib;
-    if (GATHER) {
-      ra = va ? __ldg(rows + ia) : 0;
-      rb = vb ? __ldg(rows + ib) : 0;
-      if (va && (ra < 0 || ra >= T)) { flag_status(a.status, kStatusBadIndex); va = false; }
-      if (vb && (rb < 0 || rb >= T)) { flag_status(a.status, kStatusBadIndex); vb = false; }
-      // masked lanes address row 0 (T >= 1 here), so no address leaves the sequence
-      if (!va) ra = 0;
-      if (!vb) rb = 0;
-    } else {
-      // masked lanes address the block's first row, which is < i_end <= T
-      if (!va) ra = i0;
-      if (!vb) rb = i0;
-    }
-    const uint16_t* kpa = Kb + (int64_t)ra * kHeadDim + 8 * tig;
-    const uint16_t* kpb = Kb + (int64_t)rb * kHeadDim + 8 * tig;
-    const uint16_t* vpa = Vb + (int64_t)ra * kHeadDim + 8 * tig;
-    const uint16_t* vpb = Vb + (int64_t)rb * kHeadDim + 8 * tig;
-    uint4 ka[4], kb[4], va4[4], vb4[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      ka[j] = va ? ldg_stream16(kpa + 32 * j) : make_uint4(0, 0, 0, 0);
-      kb[j] = vb ? ldg_stream16(kpb + 32 * j) : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      va4[j] = va ? ldg_stream16(vpa + 32 * j) : make_uint4(0, 0, 0, 0);
-      vb4[j] = vb ? ldg_stream16(vpb + 32 * j) : make_uint4(0, 0, 0, 0);
-    }
-
-    // S^T = K · Q^T  (rows: tokens ia / ib; cols: heads 2tig, 2tig+1)
-    float s[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int st = 0; st < 8; ++st) {
-      const int j = st >> 1, hf = st & 1;
-      mma_bf16_16816(s, word_of(ka[j], 2 * hf), word_of(kb[j], 2 * hf),
-                     word_of(ka[j], 2 * hf + 1), word_of(kb[j], 2 * hf + 1),
-                     qf[j][2 * hf], qf[j][2 * hf + 1]);
-    }
-    s[0] = va ? s[0] * a.scale_log2 : -INFINITY;
-    s[1] = va ? s[1] * a.scale_log2 : -INFINITY;
-    s[2] = vb ? s[2] * a.scale_log2 : -INFINITY;
-    s[3] = vb ? s[3] * a.scale_log2 : -INFINITY;
-
-    if (!GATHER) {
-      if (2 * tig + 1 < G) {
-        if (va) *reinterpret_cast<float2*>(lrow + (int64_t)ia * G + 2 * tig) = make_float2(s[0], s[1]);
-        if (vb) *reinterpret_cast<float2*>(lrow + (int64_t)ib * G + 2 * tig) = make_float2(s[2], s[3]);
-      } else if (2 * tig < G) {
-        if (va) lrow[(int64_t)ia * G + 2 * tig] = s[0];
-        if (vb) lrow[(int64_t)ib * G + 2 * tig] = s[2];
-      }
-    }
-
-    // online softmax (base 2)
-    const float mx0 = warp_max_xor_gid(fmaxf(s[0], s[2]));
-    const float mx1 = warp_max_xor_gid(fmaxf(s[1], s[3]));
-    const float mn0 = fmaxf(m_run0, mx0), mn1 = fmaxf(m_run1, mx1);
-    const float base0 = (mn0 == -INFINITY) ? 0.f : mn0;
-    const float base1 = (mn1 == -INFINITY) ? 0.f : mn1;
-    const float al0 = fast_exp2(m_run0 - base0), al1 = fast_exp2(m_run1 - base1);
-    const float p0 = fast_exp2(s[0] - base0), p1 = fast_exp2(s[1] - base1);
-    const float p2 = fast_exp2(s[2] - base0), p3 = fast_exp2(s[3] - base1);
-    l_run0 = l_run0 * al0 + p0 + p2;
-    l_run1 = l_run1 * al1 + p1 + p3;
-    m_run0 = mn0;
-    m_run1 = mn1;
-#pragma unroll
-    for (int mt = 0; mt < 8; ++mt) {
-      o[mt][0] *= al0; o[mt][1] *= al1; o[mt][2] *= al0; o[mt][3] *= al1;
-    }
-
-    // O^T += V^T · P^T
-    const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p0, p1));
-    const uint32_t pb1 = movmatrix_trans(pack_bf16x2(p2, p3));
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-#pragma unroll
-      for (int pp = 0; pp < 2; ++pp) {
-        const uint32_t a0 = movmatrix_trans(word_of(va4[j], 2 * pp));
-        const uint32_t a1 = movmatrix_trans(word_of(va4[j], 2 * pp + 1));
-        const uint32_t a2 = movmatrix_trans(word_of(vb4[j], 2 * pp));
-        const uint32_t a3 = movmatrix_trans(word_of(vb4[j], 2 * pp + 1));
-        mma_bf16_16816(o[2 * j + pp], a0, a1, a2, a3, pb0, pb1);
-      }
-    }
+    Blk x0;
+    load_blk<GATHER>(x0, i0, i_end, rows, T, Kb, Vb, gid, tig, a.status);
+    compute_blk<GATHER>(x0, ws, qf, a.scale_log2, lrow, G, tig);
+  }
   }
 
   // ---- merge the 4 warps of the CTA --------------------------------------
-  const float lsum0 = warp_sum_xor_gid(l_run0);
-  const float lsum1 = warp_sum_xor_gid(l_run1);
+  const float lsum0 = warp_sum_xor_gid(ws.l0);
+  const float lsum1 = warp_sum_xor_gid(ws.l1);
   if (gid == 0) {
-    sm_m[warp][2 * tig] = m_run0;
-    sm_m[warp][2 * tig + 1] = m_run1;
+    sm_m[warp][2 * tig] = ws.m0;
+    sm_m[warp][2 * tig + 1] = ws.m1;
     sm_l[warp][2 * tig] = lsum0;
     sm_l[warp][2 * tig + 1] = lsum1;
   }
@@ -236,10 +288,10 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(const SplitArgs 
 #pragma unroll
     for (int pp = 0; pp < 2; ++pp) {
       const int d0 = 8 * ((gid >> 1) + 4 * j) + 4 * pp + (gid & 1);
-      sm_o[warp][2 * tig][d0] = o[2 * j + pp][0];
-      sm_o[warp][2 * tig + 1][d0] = o[2 * j + pp][1];
-      sm_o[warp][2 * tig][d0 + 2] = o[2 * j + pp][2];
-      sm_o[warp][2 * tig + 1][d0 + 2] = o[2 * j + pp][3];
+      sm_o[warp][2 * tig][d0] = ws.o[2 * j + pp][0];
+      sm_o[warp][2 * tig + 1][d0] = ws.o[2 * j + pp][1];
+      sm_o[warp][2 * tig][d0 + 2] = ws.o[2 * j + pp][2];
+      sm_o[warp][2 * tig + 1][d0 + 2] = ws.o[2 * j + pp][3];
     }
   }
   __syncthreads();
@@ -266,6 +318,198 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(const SplitArgs 
       a.part_ml[slot * 2 + 1] = lsum;
     }
   }
+
+}
+
+// Reuse (gathered rows): each warp keeps kGStages blocks of 16 rows in its own
+// shared-memory ring, filled with 16-byte cp.async copies (each warp
+// instruction moves two whole 256-byte rows) and consumed by the same warp, so
+// the next blocks' loads are in flight while a block is computed without
+// holding them in registers.  Chunk c of row r is stored at c ^ 4(r & 1) so the
+// fragment reads (rows r, r+1 in one 8-lane phase) hit different banks.
+// Masked rows (past the count, or an index out of range) are zero-filled and
+// excluded from the softmax.
+#ifndef KASCADE_GATHER_STAGES
+#define KASCADE_GATHER_STAGES 2
+#endif
+constexpr int kGStages = KASCADE_GATHER_STAGES;
+constexpr uint32_t kGStageBytes = 16u * 512u;  // 16 K rows, then 16 V rows
+constexpr uint32_t kGSmem = kWarps * kGStages * kGStageBytes + 128;
+
+__device__ __forceinline__ uint32_t gswz(int r, int c) {
+  return (uint32_t)r * 256u + ((uint32_t)(c ^ ((r & 1) << 2)) << 4);
+}
+
+__global__ void __launch_bounds__(kThreads, 3) decode_gather_kernel(const SplitArgs a) {
+  extern __shared__ uint8_t gsm_raw[];
+  uint8_t* gsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gsm_raw) + 127) & ~uintptr_t(127));
+  __shared__ uint32_t smask[kWarps][kGStages];
+  __shared__ float sm_m[kWarps][8];
+  __shared__ float sm_l[kWarps][8];
+  __shared__ float sm_po[8][kHeadDim];  // this CTA's partial: unnormalised O, max, sum
+  __shared__ float sm_pm[8], sm_pl[8];
+
+  const int b = blockIdx.z, h = blockIdx.y, split = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gid = lane >> 2, tig = lane & 3;
+  const int G = a.G;
+
+  int T;
+  int64_t off;
+  const int32_t* rows;
+  int n_items = resolve_rows<true>(a, b, h, T, off, rows);
+  if (n_items < 0) {
+    if (threadIdx.x == 0 && split == 0) flag_status(a.status, kStatusBadIndex);
+    n_items = 0;
+  }
+  const uint16_t* Kb = a.k + off + (int64_t)h * T * kHeadDim;
+  const uint16_t* Vb = a.v + off + (int64_t)h * T * kHeadDim;
+  const int i_begin = (split * kWarps + warp) * a.tok_per_warp;
+  const int i_end = min(i_begin + a.tok_per_warp, n_items);
+  const int nblk = i_end > i_begin ? (i_end - i_begin + 15) / 16 : 0;
+  const uint32_t ring = smem_u32(gsm) + (uint32_t)warp * kGStages * kGStageBytes;
+
+  uint32_t qf[4][4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int gq = gid < G ? gid : G - 1;
+    uint4 t = ldg16(a.q + ((int64_t)b * a.Hq + h * G + gq) * kHeadDim + 8 * (tig + 4 * j));
+    if (gid >= G) t = make_uint4(0, 0, 0, 0);
+    qf[j][0] = t.x; qf[j][1] = t.y; qf[j][2] = t.z; qf[j][3] = t.w;
+  }
+
+  // lane -> (row parity, 16-byte chunk): rows 2i + (lane >> 4), chunk lane & 15
+  const int c16 = lane & 15, rpar = lane >> 4;
+  auto issue = [&](int bi) {
+    const int st = bi % kGStages;
+    const uint32_t dst = ring + (uint32_t)st * kGStageBytes;
+    // validity of the block's 16 rows (lanes 0..15), kept for the softmax mask
+    const int itv = i_begin + 16 * bi + (lane & 15);
+    bool okv = false;
+    if (itv < i_end) {
+      const int key = __ldg(rows + itv);
+      okv = key >= 0 && key < T;
+      if (!okv && lane < 16) flag_status(a.status, kStatusBadIndex);
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, okv) & 0xffffu;
+    if (lane == 0) smask[warp][st] = m;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = 2 * i + rpar;
+      const int it = i_begin + 16 * bi + r;
+      int key = it < i_end ? __ldg(rows + it) : 0;
+      const bool ok = (m >> r) & 1u;
+      if (!ok) key = 0;  // zero-filled from a valid address (T >= 1 whenever there are items)
+      const uint32_t o = gswz(r, c16);
+      cp_async16(dst + o, Kb + (int64_t)key * kHeadDim + c16 * 8, ok ? 16u : 0u);
+      cp_async16(dst + 4096u + o, Vb + (int64_t)key * kHeadDim + c16 * 8, ok ? 16u : 0u);
+    }
+  };
+
+  WarpState ws;
+  ws.m0 = ws.m1 = -INFINITY;
+  ws.l0 = ws.l1 = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) ws.o[i][0] = ws.o[i][1] = ws.o[i][2] = ws.o[i][3] = 0.f;
+
+  for (int bi = 0; bi < kGStages - 1; ++bi) {
+    if (bi < nblk) issue(bi);
+    cp_async_commit();
+  }
+  for (int bi = 0; bi < nblk; ++bi) {
+    if (bi + kGStages - 1 < nblk) issue(bi + kGStages - 1);
+    cp_async_commit();                  // one group per block (possibly empty)
+    cp_async_wait<kGStages - 1>();      // this lane's copies of block bi landed
+    __syncwarp();                       // ... and every other lane's
+    const int st = bi % kGStages;
+    const uint32_t src = ring + (uint32_t)st * kGStageBytes;
+    const uint32_t m = smask[warp][st];
+    Blk x;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int c = tig + 4 * j;
+      x.ka[j] = lds128(src + gswz(gid, c));
+      x.kb[j] = lds128(src + gswz(gid + 8, c));
+      x.va[j] = lds128(src + 4096u + gswz(gid, c));
+      x.vb[j] = lds128(src + 4096u + gswz(gid + 8, c));
+    }
+    x.oka = (m >> gid) & 1u;
+    x.okb = (m >> (gid + 8)) & 1u;
+    x.ia = x.ib = 0;
+    __syncwarp();                       // stage fully read before it is refilled
+    compute_blk<true>(x, ws, qf, a.scale_log2, nullptr, G, tig);
+  }
+  cp_async_wait<0>();
+
+  // ---- merge the 4 warps (the rings are free now) ---------------------------
+  const float lsum0 = warp_sum_xor_gid(ws.l0);
+  const float lsum1 = warp_sum_xor_gid(ws.l1);
+  __syncthreads();
+  float (*sm_o)[8][kHeadDim] = reinterpret_cast<float (*)[8][kHeadDim]>(gsm);  // 16 KB of the rings
+  if (gid == 0) {
+    sm_m[warp][2 * tig] = ws.m0;
+    sm_m[warp][2 * tig + 1] = ws.m1;
+    sm_l[warp][2 * tig] = lsum0;
+    sm_l[warp][2 * tig + 1] = lsum1;
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+#pragma unroll
+    for (int pp = 0; pp < 2; ++pp) {
+      const int d0 = 8 * ((gid >> 1) + 4 * j) + 4 * pp + (gid & 1);
+      sm_o[warp][2 * tig][d0] = ws.o[2 * j + pp][0];
+      sm_o[warp][2 * tig + 1][d0] = ws.o[2 * j + pp][1];
+      sm_o[warp][2 * tig][d0 + 2] = ws.o[2 * j + pp][2];
+      sm_o[warp][2 * tig + 1][d0 + 2] = ws.o[2 * j + pp][3];
+    }
+  }
+  __syncthreads();
+
+  // CTA partial of each head, kept in shared memory for the cluster merge
+  const int d = threadIdx.x;
+  for (int g = 0; g < G; ++g) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sm_m[w][g]);
+    float acc = 0.f, lsum = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const float f = fast_exp2(sm_m[w][g] - M);
+        acc += f * sm_o[w][g][d];
+        lsum += f * sm_l[w][g];
+      }
+    }
+    sm_po[g][d] = acc;
+    if (d == 0) {
+      sm_pm[g] = M;
+      sm_pl[g] = lsum;
+    }
+  }
+
+  // The splits of (b, h) form one thread-block cluster: rank 0 merges the
+  // others' partials through distributed shared memory.
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  cluster.sync();
+  if (cluster.block_rank() == 0) {
+    const int ns = (int)cluster.num_blocks();
+    for (int g = 0; g < G; ++g) {
+      float M = -INFINITY;
+      for (int r = 0; r < ns; ++r) M = fmaxf(M, *cluster.map_shared_rank(&sm_pm[g], r));
+      float L = 0.f, acc = 0.f;
+      if (M != -INFINITY) {
+        for (int r = 0; r < ns; ++r) {
+          const float f = fast_exp2(*cluster.map_shared_rank(&sm_pm[g], r) - M);
+          L += f * *cluster.map_shared_rank(&sm_pl[g], r);
+          acc += f * *cluster.map_shared_rank(&sm_po[g][d], r);
+        }
+      }
+      a.out[((int64_t)b * a.Hq + h * G + g) * kHeadDim + d] = to_bf16_bits(L > 0.f ? acc / L : 0.f);
+      if (a.lse && d == 0) a.lse[(int64_t)b * a.Hq + h * G + g] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
+    }
+  }
+  cluster.sync();  // peers keep their shared memory until rank 0 has read it
 }
 
 struct CombineArgs {
@@ -339,10 +583,20 @@ __global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(const C
     const float invG = 1.f / (float)G;
     if (G == 4) {
       const float l0 = s_lse2[0], l1 = s_lse2[1], l2 = s_lse2[2], l3 = s_lse2[3];
-      for (int t = t_lo + threadIdx.x; t < t_hi; t += kCombineThreads) {
-        const float4 s = *reinterpret_cast<const float4*>(lrow + (int64_t)t * 4);
-        prow[t] = (fast_exp2(s.x - l0) + fast_exp2(s.y - l1) + fast_exp2(s.z - l2) +
-                   fast_exp2(s.w - l3)) * invG;
+      constexpr int kU = kPoolChunk / kCombineThreads;  // tokens per thread, loads issued together
+      float4 sv[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int t = t_lo + threadIdx.x + u * kCombineThreads;
+        sv[u] = t < t_hi ? __ldcs(reinterpret_cast<const float4*>(lrow + (int64_t)t * 4))
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int t = t_lo + threadIdx.x + u * kCombineThreads;
+        if (t < t_hi)
+          prow[t] = (fast_exp2(sv[u].x - l0) + fast_exp2(sv[u].y - l1) + fast_exp2(sv[u].z - l2) +
+                     fast_exp2(sv[u].w - l3)) * invG;
       }
     } else {
       for (int t = t_lo + threadIdx.x; t < t_hi; t += kCombineThreads) {
@@ -358,11 +612,14 @@ struct WsLayout {
   size_t logits, part_ml, part_o, total;
 };
 
-WsLayout ws_layout(int B, int Hkv, int G, int max_T, int nsplit, bool with_logits) {
-  WsLayout w;
+// Anchor workspace: logits, then the split partials.  Reuse needs none: its
+// splits merge on chip.
+WsLayout ws_layout(int B, int Hkv, int G, int max_T, int nsplit, bool anchor) {
+  WsLayout w = {0, 0, 0, 0};
+  if (!anchor) return w;
   size_t off = 0;
   w.logits = off;
-  if (with_logits) off = align_up(off + (size_t)B * Hkv * max_T * G * sizeof(float), 256);
+  off = align_up(off + (size_t)B * Hkv * max_T * G * sizeof(float), 256);
   w.part_ml = off;
   off = align_up(off + (size_t)B * Hkv * nsplit * G * 2 * sizeof(float), 256);
   w.part_o = off;
@@ -373,30 +630,50 @@ WsLayout ws_layout(int B, int Hkv, int G, int max_T, int nsplit, bool with_logit
 
 }  // namespace
 
-DecodeSplit decode_split_for(int units, int n_items) {
-  // Largest per-warp run (<= 256 items) that still gives >= 4 CTAs per SM.
-  constexpr int kTargetCtas = 4 * 148;
-  int tpw = 256;
+#ifndef KASCADE_DECODE_TARGET_CTAS
+#define KASCADE_DECODE_TARGET_CTAS (4 * 148)
+#endif
+#ifndef KASCADE_DECODE_MAX_TPW
+#define KASCADE_DECODE_MAX_TPW 256
+#endif
+
+DecodeSplit decode_split_for(int units, int n_items, bool gather) {
+  DecodeSplit s;
+  if (gather) {
+    // One wave of the gather kernel (3 resident CTAs per SM): split each row
+    // into floor(444 / rows) CTAs (between 1 and 8), 4 warps each, 16-row blocks.
+    constexpr int kSlots = 3 * 148;
+    int nsplit = units >= kSlots ? 1 : kSlots / units;
+    if (nsplit > 8) nsplit = 8;  // the splits of a row form one (portable-size) cluster
+    int tpw = (n_items + 4 * nsplit - 1) / (4 * nsplit);
+    tpw = ((tpw + 15) / 16) * 16;
+    s.tok_per_warp = tpw > 16 ? tpw : 16;
+    s.nsplit = n_items > 0 ? (n_items + 4 * s.tok_per_warp - 1) / (4 * s.tok_per_warp) : 1;
+    return s;
+  }
+  // Largest per-warp run (<= KASCADE_DECODE_MAX_TPW items) that still gives at
+  // least KASCADE_DECODE_TARGET_CTAS CTAs.
+  constexpr int kTargetCtas = KASCADE_DECODE_TARGET_CTAS;
+  int tpw = KASCADE_DECODE_MAX_TPW;
   while (tpw > 16) {
     const int per_cta = kWarps * tpw;
     const long long ctas = (long long)units * ((n_items + per_cta - 1) / per_cta);
     if (ctas >= kTargetCtas) break;
     tpw /= 2;
   }
-  DecodeSplit s;
   s.tok_per_warp = tpw;
   s.nsplit = n_items > 0 ? (n_items + kWarps * tpw - 1) / (kWarps * tpw) : 1;
   return s;
 }
 
 size_t decode_workspace_bytes(int B, int Hkv, int G, int n_items, bool with_logits) {
-  const DecodeSplit sp = decode_split_for(B * Hkv, n_items);
+  const DecodeSplit sp = decode_split_for(B * Hkv, n_items, !with_logits);
   return ws_layout(B, Hkv, G, n_items, sp.nsplit, with_logits).total;
 }
 
 static cudaError_t launch_decode(const DecodeParams& p, bool gather, cudaStream_t st) {
   const int n_items = gather ? p.k_max : p.max_T;
-  const DecodeSplit sp = decode_split_for(p.B * p.Hkv, n_items);
+  const DecodeSplit sp = decode_split_for(p.B * p.Hkv, n_items, gather);
   const WsLayout w = ws_layout(p.B, p.Hkv, p.G, n_items, sp.nsplit, !gather);
   char* ws = static_cast<char*>(p.ws);
 
@@ -408,15 +685,34 @@ static cudaError_t launch_decode(const DecodeParams& p, bool gather, cudaStream_
   a.nsplit = sp.nsplit;
   a.scale_log2 = (float)((double)p.scale * 1.4426950408889634);
   a.logits = gather ? nullptr : reinterpret_cast<float*>(ws + w.logits);
-  a.part_ml = reinterpret_cast<float*>(ws + w.part_ml);
-  a.part_o = reinterpret_cast<float*>(ws + w.part_o);
+  a.part_ml = gather ? nullptr : reinterpret_cast<float*>(ws + w.part_ml);
+  a.part_o = gather ? nullptr : reinterpret_cast<float*>(ws + w.part_o);
+  a.out = p.out;
+  a.lse = p.lse;
   a.status = p.status;
 
   dim3 grid(sp.nsplit, p.Hkv, p.B);
-  if (gather)
-    decode_split_kernel<true><<<grid, kThreads, 0, st>>>(a);
-  else
-    decode_split_kernel<false><<<grid, kThreads, 0, st>>>(a);
+  if (gather) {
+    // reuse: the nsplit CTAs of each (b, h) are one cluster and merge on chip
+    cudaError_t e = cudaFuncSetAttribute(decode_gather_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGSmem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kGSmem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = sp.nsplit;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, decode_gather_kernel, a);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
+  decode_split_kernel<false><<<grid, kThreads, 0, st>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
@@ -427,7 +723,7 @@ static cudaError_t launch_decode(const DecodeParams& p, bool gather, cudaStream_
   c.logits = a.logits;
   c.pooled = p.pooled; c.ld_pooled = p.ld_pooled;
   c.out = p.out; c.lse = p.lse;
-  const int nchunk = gather ? 1 : max(1, (p.max_T + kPoolChunk - 1) / kPoolChunk);
+  const int nchunk = max(1, (p.max_T + kPoolChunk - 1) / kPoolChunk);
   dim3 cgrid(nchunk, p.Hkv, p.B);
   decode_combine_kernel<<<cgrid, kCombineThreads, 0, st>>>(c);
   return cudaGetLastError();

@@ -38,7 +38,7 @@ struct DecodeSplit {
   int tok_per_warp;
   int nsplit;  // CTAs per (b, h)
 };
-DecodeSplit decode_split_for(int units, int n_items);
+DecodeSplit decode_split_for(int units, int n_items, bool gather);
 size_t decode_workspace_bytes(int B, int Hkv, int G, int n_items, bool with_logits);
 
 cudaError_t launch_decode_anchor(const DecodeParams& p, cudaStream_t st);

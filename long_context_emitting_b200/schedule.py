@@ -145,7 +145,7 @@ class PrefillSchedule:
 # Kernel launches issued by one call of each entry point.
 LAUNCHES = {
     "decode_anchor": 2,   # split-K attention, combine + pooled
-    "decode_reuse": 2,    # split-K gathered attention, combine
+    "decode_reuse": 1,    # gathered attention; the splits of a row merge in a thread-block cluster
     "topk": 1,
     "prefill_anchor": 2,  # causal attention (O, LSE), pooled probabilities
     "prefill_reuse": 1,
@@ -160,3 +160,30 @@ def launches_per_step(dec: "DecodeSchedule | None", pre: "PrefillSchedule | None
         for l in range(sch.n_layers):
             n += LAUNCHES[a] + LAUNCHES["topk"] if sch.is_anchor(l) else LAUNCHES[r]
     return n
+
+
+class StepGraph:
+    """A whole schedule step (every layer's launches) captured as one CUDA graph.
+
+    The schedules preallocate all buffers, so a step issues kernel launches
+    only; capturing it removes the per-launch host cost between layers.
+    Inputs are read from the tensors that were passed at capture time: update
+    them in place (e.g. copy the new queries into ``layers[l]["q"]``) and
+    ``replay()``.
+    """
+
+    def __init__(self, step_fn, warmup: int = 1):
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for _ in range(warmup):   # first calls cache kernel attributes and tensor-map encoders
+                step_fn()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            step_fn()
+        torch.cuda.synchronize()
+
+    def replay(self):
+        self.graph.replay()

@@ -81,10 +81,8 @@ def test_workspace_too_small(lib):
     assert need > 4 * 8 * 32768 * 16  # holds the per-head logits
     assert lib.kascade_decode_anchor(s, P, P, P, P, P, 32768, 0.1, P, P, P, 32768, P, need - 1,
                                      None) == WS_SMALL
-    need_r = lib.kascade_decode_reuse_workspace_bytes(s, 3277)
-    assert need_r > 0
-    assert lib.kascade_decode_reuse(s, P, P, P, P, P, P, P, 3277, P, 0.1, P, P, P, need_r - 1,
-                                    None) == WS_SMALL
+    # reuse merges its splits on chip (thread-block clusters): no workspace
+    assert lib.kascade_decode_reuse_workspace_bytes(s, 3277) == 0
 
 
 def test_empty_batch_is_a_no_op(lib):
