@@ -15,7 +15,7 @@ CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libkascade.so")
 SOURCES = ["api.cu", "decode.cu", "topk.cu", "prefill.cu", "noalloc.cu"]
-HEADERS = ["common.cuh", "internal.h", "tcgen05.cuh"]
+HEADERS = ["common.cuh", "internal.h", "tcgen05.cuh", "exp2_poly.cuh", "f32x2.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
