@@ -23,8 +23,9 @@
  *   - Errors found by the kernels themselves (an index, head-map entry or length
  *     out of range, a NaN score) never fault: the offending element is skipped, and
  *     a sticky per-device status word is set; read it with kascade_get_device_status.
- *   - Supported shapes: head_dim d == 128, Hq % Hkv == 0, group size Hq/Hkv <= 8,
+ *   - Supported shapes: head_dim d == 128, Hq % Hkv == 0, group size Hq/Hkv in {1,2,4,8},
  *     prefill query tile fixed at 128 tokens, prefill length a multiple of 128.
+ *   - `scale` must be finite; the prefill calls also require scale > 0.
  *   - Returned status codes are the kascade_status values below; no C++ exception
  *     crosses this boundary.
  */

@@ -187,7 +187,7 @@ int kascade_prefill_anchor(kascade_shape s, int32_t N, const uint16_t* q, const 
                            float* pooled, void* ws, size_t ws_bytes, void* stream) {
   int rc = check_prefill(s, N);
   if (rc) return rc;
-  if (!std::isfinite(scale)) return KASCADE_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return KASCADE_ERR_INVALID_ARG;
   if (s.B == 0 || N == 0) return KASCADE_OK;
   const size_t need = kascade_prefill_anchor_workspace_bytes(s, N);
   if (!q || !k || !v || !out || !lse || !pooled || (need && !ws)) return KASCADE_ERR_INVALID_ARG;
@@ -217,7 +217,7 @@ int kascade_prefill_reuse(kascade_shape s, int32_t N, const uint16_t* q, const u
                           float* lse, void* ws, size_t ws_bytes, void* stream) {
   int rc = check_prefill(s, N);
   if (rc) return rc;
-  if (k_max < 0 || !std::isfinite(scale)) return KASCADE_ERR_INVALID_ARG;
+  if (k_max < 0 || !std::isfinite(scale) || !(scale > 0.f)) return KASCADE_ERR_INVALID_ARG;
   if (s.B == 0 || N == 0) return KASCADE_OK;
   const size_t need = kascade_prefill_reuse_workspace_bytes(s, N, k_max);
   if (!q || !k || !v || !idx || !idx_k || !head_map || !out || (need && !ws))

@@ -9,37 +9,43 @@
 // prefill_attn_kernel<GATHER>
 //   One CTA per (query tile t, pair of query heads of one GQA group, sequence).
 //   The two heads share every K/V block, so each block is loaded once for two
-//   128 x 128 attention tiles.  Warp roles (384 threads):
-//     warp 0      TMA producer: Q tiles, then K/V blocks into a 2-stage ring.
+//   128 x 128 attention tiles.  Warp roles (384 threads, three warpgroups):
+//     warp 8      TMA producer: Q tiles, then K/V blocks into a 2-stage ring.
 //                 anchor: dense key blocks 0..t (block t is the diagonal);
 //                 reuse: the anchor's indices of row (t, head_map[h]) gathered
 //                 with cp.async (two whole rows per warp instruction) into the
 //                 same swizzled layout, then the diagonal block by TMA.
-//     warp 1      MMA issuer (one thread): S_i = Q_i K^T into TMEM, and
+//     warp 9      MMA issuer (one thread): S_i = Q_i K^T into TMEM, and
 //                 O_i += P_i V with P_i read from TMEM (it overwrites S_i).
-//     warps 4-7   softmax of tile 0, warps 8-11 softmax of tile 1: thread r
-//                 owns query row r (TMEM lane r), reads S, runs the online
-//                 softmax in base 2 (the running maximum is raised only when a
-//                 block exceeds it by 2^8, so O is rarely rescaled), writes P
-//                 back to TMEM as bf16 and finally normalises O.
+//     warps 0-7   softmax, one warpgroup per tile, one query row (TMEM lane)
+//                 per thread: the row's 128 scores are loaded into registers
+//                 at once, so the row maximum needs no exchange between
+//                 threads.  Online softmax in base 2 (the running maximum is
+//                 raised only when a block exceeds it by 2^8, so O is rarely
+//                 rescaled); P goes back to TMEM as bf16 over the row's S.
 //   The MMA thread alternates between the tiles, so the tensor cores work on
-//   one tile while the other tile's softmax runs.
+//   one tile while the other tile's softmax runs.  The softmax warpgroups take
+//   registers from the third one (setmaxnreg; the launch checks the split).
 //   TMEM (512 columns): S0|P0 [0,128), O0 [128,256), S1|P1 [256,384), O1 [384,512).
 //
 // prefill_pool_kernel
 //   One CTA per (tile t >= 1, KV head, sequence).  For each key block before
 //   the tile it computes S^T = K Q_g^T for the group's query heads (keys on
 //   TMEM lanes, queries on columns), so a thread owns one key and sums
-//   exp2(s - lse2) over the tile's queries in registers.  Warp roles: a TMA
+//   exp2(s - lse2) over the tile's queries in registers (3 of 8 exponentials
+//   on the FMA pipe, the rest on the SFU).  Warp roles: a TMA
 //   producer, an MMA issuer and two warpgroups that each sum half of the heads
 //   (ping-ponging on two TMEM regions); the two halves are added through shared
 //   memory and pooled = sum / (128 G) is written once, without atomics.
+#include "exp2_poly.cuh"
+#include "f32x2.cuh"
 #include "tcgen05.cuh"
 #include "internal.h"
 
 #include <cudaTypedefs.h>
 
 #include <cmath>
+
 
 namespace kascade {
 
@@ -53,7 +59,15 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ---- attention kernel layout ----
-constexpr int kAttnThreads = 384;
+constexpr int kAttnThreads = 384;  // softmax warps 0-7, producer warp 8, MMA warp 9 (10, 11 idle)
+constexpr int kProducerWarp = 8, kMmaWarp = 9;
+// setmaxnreg split: the launch gives every thread kLaunchRegs (the compiler's
+// count, checked on the host); the third warpgroup releases down to kOtherRegs
+// and the two softmax warpgroups take exactly what it releases.
+constexpr int kLaunchRegs = 168, kSoftmaxRegs = 200, kOtherRegs = 104;
+static_assert((kLaunchRegs - kOtherRegs) * 128 >= (kSoftmaxRegs - kLaunchRegs) * 256,
+              "softmax register increase must fit in what the third warpgroup releases");
+static_assert(kLaunchRegs * kAttnThreads <= 65536, "launch registers exceed the SM");
 constexpr uint32_t kAttnQ = 0;                         // 2 query tiles
 constexpr uint32_t kAttnKV = 2 * kTileBytes;           // stage s: K at +2s*tile, V at +(2s+1)*tile
 constexpr uint32_t kAttnMisc = kAttnKV + 4 * kTileBytes;
@@ -100,6 +114,14 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int ks) {
 __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile, int ks) {
   return sw128_desc(tile + (uint32_t)ks * 2048u, kHalfBytes, 1024u);
 }
+// The start-address field is the low 14 bits of (address >> 4); shared
+// addresses stay below 2^18, so a k-step is a constant added to a base
+// descriptor (no carry out of the field).  Saves the MMA-issuing thread, which
+// shares its scheduler with busy softmax warps, most of its instructions.
+__device__ __forceinline__ constexpr uint64_t kmajor_step(int ks) {
+  return (uint64_t)(((uint32_t)(ks >> 2) * kHalfBytes + (uint32_t)(ks & 3) * 32u) >> 4);
+}
+__device__ __forceinline__ constexpr uint64_t mnmajor_step(int ks) { return (uint64_t)(ks * 2048u >> 4); }
 
 __device__ __forceinline__ volatile int* abort_flag(uint8_t* smem, uint32_t misc) {
   return reinterpret_cast<volatile int*>(smem + misc + 128);
@@ -112,10 +134,11 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kAttnMisc);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kAttnMisc + 96);
-  volatile int* s_abort = abort_flag(smem, kAttnMisc);
-  uint32_t* masks = reinterpret_cast<uint32_t*>(smem + kAttnMisc + 160);  // [2 stages][4]
+  uint8_t* misc = smem + kAttnMisc;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(misc);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 128);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(misc + 136);
+  uint32_t* masks = reinterpret_cast<uint32_t*>(misc + 160);        // [2 stages][4]
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -148,11 +171,14 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   const int kv_row0 = (int)(((int64_t)b * a.Hkv + h) * a.N);
 
   if (tid == 0) {
-    for (int i = 0; i < kAttnBars; ++i) mbar_init(bar(i), (i == kBarP || i == kBarP + 1) ? 128u : 1u);
+    for (int i = 0; i < kAttnBars; ++i) {
+      const bool per_warp = i >= kBarP && i < kBarP + 2;  // 4 softmax warps per tile
+      mbar_init(bar(i), per_warp ? 4u : 1u);
+    }
     *s_abort = 0;
     mbar_fence_init();
   }
-  if (warp == 2) {
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
@@ -161,134 +187,146 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ================================ TMA producer ================================
-    if (lane == 0) {
-      mbar_expect_tx(bar(kBarQ), ntile * kTileBytes);
-      for (int i = 0; i < ntile; ++i) {
-        const int y = (int)(q_row0 + (int64_t)i * a.N);
-        tma_load_2d(sbase + kAttnQ + i * kTileBytes, &tm_q, 0, y, bar(kBarQ));
-        tma_load_2d(sbase + kAttnQ + i * kTileBytes + kHalfBytes, &tm_q, 64, y, bar(kBarQ));
-      }
-    }
-    for (int j = 0; j < nblk; ++j) {
-      const int st = j & 1;
-      if (j >= 2 && !mbar_wait(bar(kBarKvEmpty + st), ((j >> 1) - 1) & 1, a.status)) { *s_abort = 1; break; }
-      if (*s_abort) break;
-      const uint32_t kb = sbase + kAttnKV + (2 * st) * kTileBytes;
-      const uint32_t vb = kb + kTileBytes;
-      const bool dense = !GATHER || j == n_gather;
-      if (dense) {
-        if (lane == 0) {
-          mbar_expect_tx(bar(kBarKvFull + st), 2 * kTileBytes);
-          const int y = kv_row0 + kTile * (GATHER ? t : j);
-          tma_load_2d(kb, &tm_k, 0, y, bar(kBarKvFull + st));
-          tma_load_2d(kb + kHalfBytes, &tm_k, 64, y, bar(kBarKvFull + st));
-          tma_load_2d(vb, &tm_v, 0, y, bar(kBarKvFull + st));
-          tma_load_2d(vb + kHalfBytes, &tm_v, 64, y, bar(kBarKvFull + st));
-        }
-      } else {
-        // Gathered block: validity of rows 4*lane .. 4*lane+3 -> 4 ballot words.
-        uint32_t m[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int pos = kTile * j + 4 * lane + e;
-          const int key = pos < kt ? __ldg(irow + pos) : -1;
-          const bool ok = key >= 0 && key < kTile * t;
-          if (pos < kt && !ok) flag_status(a.status, kStatusBadIndex);
-          m[e] = __ballot_sync(0xffffffffu, ok);
-        }
-        // Copy: each warp instruction moves two whole 256-byte rows (16 lanes per
-        // row, one 16-byte chunk each) into the swizzled layout; masked rows are
-        // zero-filled from a valid address.
-        const int c16 = lane & 15;
-        const uint32_t half = (uint32_t)(c16 >> 3) * kHalfBytes;
-        for (int s2 = 0; s2 < kTile / 2; ++s2) {
-          const int row = 2 * s2 + (lane >> 4);
-          const int pos = kTile * j + row;
-          const int key = pos < kt ? __ldg(irow + pos) : -1;
-          const bool ok = key >= 0 && key < kTile * t;
-          const int64_t src = (int64_t)kv_row0 + (ok ? key : kTile * t);
-          const uint32_t off = half + (uint32_t)row * 128u + ((uint32_t)((c16 & 7) ^ (row & 7)) << 4);
-          cp_async16(kb + off, a.k + src * kHeadDim + c16 * 8, ok ? 16u : 0u);
-          cp_async16(vb + off, a.v + src * kHeadDim + c16 * 8, ok ? 16u : 0u);
-        }
-        cp_async_commit();
-        cp_async_wait<0>();
-        fence_proxy_async_smem();  // the tensor cores read these rows through the async proxy
-        __syncwarp();
-        if (lane == 0) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) masks[st * 4 + e] = m[e];
-          mbar_arrive(bar(kBarKvFull + st));  // release: rows and masks visible
+  if (warp >= 8) {
+    setmaxnreg_dec<kOtherRegs>();
+  if (warp == kProducerWarp) {
+      // ================================ TMA producer ================================
+      if (lane == 0) {
+        mbar_expect_tx(bar(kBarQ), ntile * kTileBytes);
+        for (int i = 0; i < ntile; ++i) {
+          const int y = (int)(q_row0 + (int64_t)i * a.N);
+          tma_load_2d(sbase + kAttnQ + i * kTileBytes, &tm_q, 0, y, bar(kBarQ));
+          tma_load_2d(sbase + kAttnQ + i * kTileBytes + kHalfBytes, &tm_q, 64, y, bar(kBarQ));
         }
       }
-    }
-  } else if (warp == 1) {
-    // ================================ MMA issuer ==================================
-    if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16(128, 128, false, false);
-      const uint32_t idesc_o = idesc_bf16(128, 128, false, true);
-      auto issue_s = [&](int i, uint32_t kb) {
-        const uint32_t qs = sbase + kAttnQ + i * kTileBytes;
-#pragma unroll
-        for (int k16 = 0; k16 < 8; ++k16)
-          umma_ss(tmem + 256 * i, kmajor_desc(qs, k16), kmajor_desc(kb, k16), idesc_s, k16 > 0 ? 1u : 0u);
-      };
-      auto issue_pv = [&](int i, uint32_t vb, bool acc) {
-#pragma unroll
-        for (int k16 = 0; k16 < 8; ++k16)
-          umma_ts(tmem + 256 * i + 128, tmem + 256 * i + 8 * k16, mnmajor_desc(vb, k16), idesc_o,
-                  (acc || k16 > 0) ? 1u : 0u);
-      };
-      bool ok = mbar_wait(bar(kBarQ), 0, a.status);
-      for (int j = 0; ok && j < nblk; ++j) {
+      for (int j = 0; j < nblk; ++j) {
         const int st = j & 1;
+        if (j >= 2 && !mbar_wait(bar(kBarKvEmpty + st), ((j >> 1) - 1) & 1, a.status)) { *s_abort = 1; break; }
+        if (*s_abort) break;
         const uint32_t kb = sbase + kAttnKV + (2 * st) * kTileBytes;
         const uint32_t vb = kb + kTileBytes;
-        if (!(ok = mbar_wait(bar(kBarKvFull + st), (j >> 1) & 1, a.status))) break;
-        tc_fence_after();
-        if (j == 0) {
-          for (int i = 0; i < ntile; ++i) {
-            issue_s(i, kb);
-            umma_commit(bar(kBarS + i));
+        const bool dense = !GATHER || j == n_gather;
+        if (dense) {
+          if (lane == 0) {
+            mbar_expect_tx(bar(kBarKvFull + st), 2 * kTileBytes);
+            const int y = kv_row0 + kTile * (GATHER ? t : j);
+            tma_load_2d(kb, &tm_k, 0, y, bar(kBarKvFull + st));
+            tma_load_2d(kb + kHalfBytes, &tm_k, 64, y, bar(kBarKvFull + st));
+            tma_load_2d(vb, &tm_v, 0, y, bar(kBarKvFull + st));
+            tma_load_2d(vb + kHalfBytes, &tm_v, 64, y, bar(kBarKvFull + st));
+          }
+        } else {
+          // Gathered block: validity of rows 32e + lane -> ballot word e (bit = row & 31).
+          uint32_t m[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int pos = kTile * j + 32 * e + lane;
+            const int key = pos < kt ? __ldg(irow + pos) : -1;
+            const bool ok = key >= 0 && key < kTile * t;
+            if (pos < kt && !ok) flag_status(a.status, kStatusBadIndex);
+            m[e] = __ballot_sync(0xffffffffu, ok);
+          }
+          // Copy: each warp instruction moves two whole 256-byte rows (16 lanes per
+          // row, one 16-byte chunk each) into the swizzled layout; masked rows are
+          // zero-filled from a valid address.
+          const int c16 = lane & 15;
+          const uint32_t half = (uint32_t)(c16 >> 3) * kHalfBytes;
+          for (int s2 = 0; s2 < kTile / 2; ++s2) {
+            const int row = 2 * s2 + (lane >> 4);
+            const int pos = kTile * j + row;
+            const int key = pos < kt ? __ldg(irow + pos) : -1;
+            const bool ok = key >= 0 && key < kTile * t;
+            const int64_t src = (int64_t)kv_row0 + (ok ? key : kTile * t);
+            const uint32_t off = half + (uint32_t)row * 128u + ((uint32_t)((c16 & 7) ^ (row & 7)) << 4);
+            cp_async16(kb + off, a.k + src * kHeadDim + c16 * 8, ok ? 16u : 0u);
+            cp_async16(vb + off, a.v + src * kHeadDim + c16 * 8, ok ? 16u : 0u);
+          }
+          cp_async_commit();
+          cp_async_wait<0>();
+          fence_proxy_async_smem();  // the tensor cores read these rows through the async proxy
+          __syncwarp();
+          if (lane == 0) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) masks[st * 4 + e] = m[e];
+            mbar_arrive(bar(kBarKvFull + st));  // release: rows and masks visible
           }
         }
-        const bool more = j + 1 < nblk;
-        const uint32_t kb2 = sbase + kAttnKV + (2 * (st ^ 1)) * kTileBytes;
-        // tile 0: PV of this block, then S of the next block
-        if (!(ok = mbar_wait(bar(kBarP + 0), j & 1, a.status))) break;
-        tc_fence_after();
-        issue_pv(0, vb, j > 0);
-        if (more) {
-          if (!(ok = mbar_wait(bar(kBarKvFull + (st ^ 1)), ((j + 1) >> 1) & 1, a.status))) break;
-          tc_fence_after();
-          issue_s(0, kb2);
-          umma_commit(bar(kBarS + 0));
-        }
-        if (ntile == 2) {
-          if (!(ok = mbar_wait(bar(kBarP + 1), j & 1, a.status))) break;
-          tc_fence_after();
-          issue_pv(1, vb, j > 0);
-        }
-        umma_commit(bar(kBarKvEmpty + st));  // K/V stage free once these MMAs complete
-        if (ntile == 2 && more) {
-          issue_s(1, kb2);
-          umma_commit(bar(kBarS + 1));
-        }
-        if (*s_abort) { ok = false; break; }
       }
-      if (!ok) *s_abort = 1;
-      for (int i = 0; i < ntile; ++i) umma_commit(bar(kBarO + i));
+    } else if (warp == kMmaWarp) {
+      // ================================ MMA issuer ==================================
+      if (lane == 0) {
+        const uint32_t idesc_s = idesc_bf16(128, 128, false, false);
+        const uint32_t idesc_o = idesc_bf16(128, 128, false, true);
+        // base descriptors: query tiles, and K / V of the two stages
+        const uint64_t dq0 = kmajor_desc(sbase + kAttnQ, 0);
+        const uint64_t dq1 = kmajor_desc(sbase + kAttnQ + kTileBytes, 0);
+        const uint64_t dk0 = kmajor_desc(sbase + kAttnKV, 0);
+        const uint64_t dk1 = kmajor_desc(sbase + kAttnKV + 2 * kTileBytes, 0);
+        const uint64_t dv0 = mnmajor_desc(sbase + kAttnKV + kTileBytes, 0);
+        const uint64_t dv1 = mnmajor_desc(sbase + kAttnKV + 3 * kTileBytes, 0);
+        auto issue_s = [&](int i, int st) {
+          const uint64_t dq = i ? dq1 : dq0, dk = st ? dk1 : dk0;
+          const uint32_t d = tmem + 256 * i;
+#pragma unroll
+          for (int k16 = 0; k16 < 8; ++k16)
+            umma_ss(d, dq + kmajor_step(k16), dk + kmajor_step(k16), idesc_s, k16 > 0 ? 1u : 0u);
+        };
+        // P (128 keys as bf16 pairs) sits in columns 0..63 of the tile's S region.
+        auto issue_pv = [&](int i, int st, bool acc) {
+          const uint64_t dv = st ? dv1 : dv0;
+          const uint32_t d = tmem + 256 * i + 128, pa = tmem + 256 * i;
+#pragma unroll
+          for (int k16 = 0; k16 < 8; ++k16)
+            umma_ts(d, pa + 8 * k16, dv + mnmajor_step(k16), idesc_o, (acc || k16 > 0) ? 1u : 0u);
+        };
+        bool ok = mbar_wait(bar(kBarQ), 0, a.status);
+        for (int j = 0; ok && j < nblk; ++j) {
+          const int st = j & 1;
+          if (!(ok = mbar_wait(bar(kBarKvFull + st), (j >> 1) & 1, a.status))) break;
+          tc_fence_after();
+          if (j == 0) {
+            for (int i = 0; i < ntile; ++i) {
+              issue_s(i, st);
+              umma_commit(bar(kBarS + i));
+            }
+          }
+          const bool more = j + 1 < nblk;
+          // tile 0: PV of this block, then S of the next block
+          if (!(ok = mbar_spin(bar(kBarP + 0), j & 1, a.status))) break;
+          tc_fence_after();
+          issue_pv(0, st, j > 0);
+          if (more) {
+            if (!(ok = mbar_wait(bar(kBarKvFull + (st ^ 1)), ((j + 1) >> 1) & 1, a.status))) break;
+            tc_fence_after();
+            issue_s(0, st ^ 1);
+            umma_commit(bar(kBarS + 0));
+          }
+          if (ntile == 2) {
+            if (!(ok = mbar_spin(bar(kBarP + 1), j & 1, a.status))) break;
+            tc_fence_after();
+            issue_pv(1, st, j > 0);
+          }
+          umma_commit(bar(kBarKvEmpty + st));  // K/V stage free once these MMAs complete
+          if (ntile == 2 && more) {
+            issue_s(1, st ^ 1);
+            umma_commit(bar(kBarS + 1));
+          }
+          if (*s_abort) { ok = false; break; }
+        }
+        if (!ok) *s_abort = 1;
+        for (int i = 0; i < ntile; ++i) umma_commit(bar(kBarO + i));
+      }
     }
-  } else if (warp >= 4) {
+  } else {
+    setmaxnreg_inc<kSoftmaxRegs>();
     // ================================ softmax =====================================
-    const int i = (warp - 4) >> 2;  // tile
-    const int r = tid - 128 - 128 * i;  // query row = TMEM lane
+    // Warpgroup i handles tile i; thread = query row r = TMEM lane.
+    const int i = warp >> 2;
+    const int r = (warp & 3) * 32 + lane;
     if (i < ntile) {
-      const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-      const uint32_t tS = tmem + 256 * i + lane_base;
+      const uint32_t tS = tmem + 256 * i + ((uint32_t)((warp & 3) * 32) << 16);  // S (and P)
       const uint32_t tO = tS + 128;
+      const float sc = a.scale_log2;  // > 0, so max(s) * sc = max(s * sc)
       float m_used = -INFINITY, l_sum = 0.f;
       bool ok = true;
       for (int j = 0; j < nblk; ++j) {
@@ -297,38 +335,59 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const bool diag = GATHER ? (j == n_gather) : (j == t);
         uint32_t mk[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
         if (GATHER && !diag) {
+          // masks of the gathered rows (written before the stage's full barrier completed)
           if (!(ok = mbar_wait(bar(kBarKvFull + (j & 1)), (j >> 1) & 1, a.status))) break;
 #pragma unroll
           for (int e = 0; e < 4; ++e) mk[e] = masks[(j & 1) * 4 + e];
         }
-        uint32_t sr[128];
+        if (diag) {
+          // causal diagonal block: key col is visible to row r if col <= r
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
-        tmem_wait_ld();
-        float mloc = -INFINITY;
-#pragma unroll
-        for (int col = 0; col < 128; ++col) {
-          bool keep = diag ? (col <= r) : (((mk[col & 3] >> (col >> 2)) & 1u) != 0u);
-          const float x = keep ? __uint_as_float(sr[col]) * a.scale_log2 : -INFINITY;
-          sr[col] = __float_as_uint(x);
-          mloc = fmaxf(mloc, x);
+          for (int c = 0; c < 4; ++c) {
+            const int n = r - 32 * c + 1;  // visible keys of this chunk
+            mk[c] = n >= 32 ? 0xffffffffu : (n <= 0 ? 0u : (1u << n) - 1u);
+          }
         }
+        uint32_t v[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, v[c]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) reg_fence32(v[c]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (mk[c] != 0xffffffffu) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (!((mk[c] >> e) & 1u)) v[c][e] = __float_as_uint(-INFINITY);
+          }
+        }
+        // ---- row maximum of the raw scores
+        float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int e2 = 0; e2 < 16; ++e2)
+            mp[e2 & 3] = fmax3(mp[e2 & 3], __uint_as_float(v[c][2 * e2]), __uint_as_float(v[c][2 * e2 + 1]));
+        const float mr = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
+        const float mloc = mr == -INFINITY ? -INFINITY : mr * sc;
         float alpha = 1.f;
         bool rescale = false;
         if (m_used == -INFINITY) {
-          m_used = mloc;
+          m_used = mloc;  // first visible key of the row: O and l are still zero
         } else if (mloc > m_used + kRescaleLog2) {
           alpha = fast_exp2(m_used - mloc);
           m_used = mloc;
           rescale = true;
         }
-        if (__any_sync(0xffffffffu, rescale) && j > 0) {
+        if (__any_sync(0xffffffffu, rescale)) {
           // the previous PV of this tile completed before S of this block was committed
 #pragma unroll 1
           for (int c = 0; c < 4; ++c) {
             uint32_t o[32];
             tmem_ld32(tO + 32 * c, o);
             tmem_wait_ld();
+            reg_fence32(o);
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
             tmem_st32(tO + 32 * c, o);
@@ -336,22 +395,35 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         l_sum *= alpha;
         const float base = (m_used == -INFINITY) ? 0.f : m_used;
-        uint32_t pw[64];
+        // ---- p = exp2(s*sc - base), two scores per packed f32x2 FMA; P goes
+        // back as bf16 pairs into columns 0..63 of the row's S (all read).
+        uint64_t L[4] = {0ull, 0ull, 0ull, 0ull};
+        const uint64_t SC = f2_pack(sc, sc), NB = f2_pack(-base, -base);
 #pragma unroll
-        for (int c2 = 0; c2 < 64; ++c2) {
-          const float p0 = fast_exp2(__uint_as_float(sr[2 * c2]) - base);
-          const float p1 = fast_exp2(__uint_as_float(sr[2 * c2 + 1]) - base);
-          l_sum += p0 + p1;
-          pw[c2] = pack_bf16x2(p0, p1);
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pw[16];
+#pragma unroll
+          for (int e2 = 0; e2 < 16; ++e2) {
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(v[c][2 * e2]), __uint_as_float(v[c][2 * e2 + 1])), SC, NB),
+                      x0, x1);
+            const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+            L[e2 & 3] = f2_add(L[e2 & 3], f2_pack(p0, p1));
+            pw[e2] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(tS + 16 * c, pw);
         }
-        tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pw[0]));
-        tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pw[32]));
+        float l0, l1, l2, l3;
+        f2_unpack(f2_add(L[0], L[1]), l0, l1);
+        f2_unpack(f2_add(L[2], L[3]), l2, l3);
+        l_sum += (l0 + l1) + (l2 + l3);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(kBarP + i));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kBarP + i));  // one arrival per warp, 4 per tile
       }
       if (!ok) *s_abort = 1;
-      // ---- epilogue: O / l ----------------------------------------------------
+      // ---- epilogue: O / l --------------------------------------------------------
       if (mbar_wait(bar(kBarO + i), 0, a.status) && ok && !*s_abort) {
         tc_fence_after();
         const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
@@ -362,6 +434,7 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           uint32_t o[32];
           tmem_ld32(tO + 32 * c, o);
           tmem_wait_ld();
+          reg_fence32(o);
 #pragma unroll
           for (int q8 = 0; q8 < 4; ++q8) {
             uint4 w;
@@ -378,7 +451,7 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 2) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -425,10 +498,10 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   for (int rd = 0; rd < n_rounds; ++rd) {
     const int hg = min(kPoolHeads, G - rd * kPoolHeads);  // heads this round
     const int gbase = h * G + rd * kPoolHeads;
-    // lse of the round's heads (log2 domain), read by the summing warps
+    // -lse of the round's heads (log2 domain), read in pairs by the summing warps
     for (int e = tid; e < hg * kTile; e += kPoolThreads) {
       const int j = e / kTile, q = e % kTile;
-      lse2[e] = a.lse[((int64_t)b * a.Hq + gbase + j) * a.N + (int64_t)kTile * t + q] * kLog2e;
+      lse2[e] = -a.lse[((int64_t)b * a.Hq + gbase + j) * a.N + (int64_t)kTile * t + q] * kLog2e;
     }
     __syncthreads();
     const int it0 = rd * nblk;  // running block counter for stage / phase bookkeeping
@@ -459,17 +532,17 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         for (int jb = 0; ok && jb < nblk; ++jb) {
           const int it = it0 + jb, st = it & 1;
           if (!(ok = mbar_wait(bar(kPBarKFull + st), (it >> 1) & 1, a.status))) break;
-          const uint32_t ks = sbase + kPoolK + st * kTileBytes;
+          const uint64_t dk = kmajor_desc(sbase + kPoolK + st * kTileBytes, 0);
           for (int w = 0; w < 2; ++w) {
             // region w holds heads 2w, 2w+1 of the round; wait until its summing
             // warpgroup has read the previous block
-            if (it >= 1 && !(ok = mbar_wait(bar(kPBarFree + w), (it - 1) & 1, a.status))) break;
+            if (it >= 1 && !(ok = mbar_spin(bar(kPBarFree + w), (it - 1) & 1, a.status))) break;
             tc_fence_after();
             for (int jj = 2 * w; jj < min(2 * w + 2, hg); ++jj) {
-              const uint32_t qs = sbase + kPoolQ + jj * kTileBytes;
+              const uint64_t dq = kmajor_desc(sbase + kPoolQ + jj * kTileBytes, 0);
 #pragma unroll
               for (int k16 = 0; k16 < 8; ++k16)
-                umma_ss(tmem + 128 * jj, kmajor_desc(ks, k16), kmajor_desc(qs, k16), idesc,
+                umma_ss(tmem + 128 * jj, dk + kmajor_step(k16), dq + kmajor_step(k16), idesc,
                         k16 > 0 ? 1u : 0u);
             }
             umma_commit(bar(kPBarS + w));
@@ -489,19 +562,38 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const int it = it0 + jb;
         if (!mbar_wait(bar(kPBarS + w), it & 1, a.status) || *s_abort) { *s_abort = 1; break; }
         tc_fence_after();
-        float acc = 0.f;
+        // sum over the queries of exp2(s * sc - lse2), two per packed instruction
+        uint64_t A[4] = {0ull, 0ull, 0ull, 0ull};
+        const uint64_t SC = f2_pack(a.scale_log2, a.scale_log2);
         for (int jj = 2 * w; jj < min(2 * w + 2, hg); ++jj) {
-          const float* l2 = lse2 + jj * kTile;
+          const uint64_t* nl2 = reinterpret_cast<const uint64_t*>(lse2 + jj * kTile);
 #pragma unroll 1
           for (int c = 0; c < 4; ++c) {
             uint32_t sv[32];
             tmem_ld32(tmem + 128 * jj + lane_base + 32 * c, sv);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-              acc += fast_exp2(__uint_as_float(sv[e]) * a.scale_log2 - l2[32 * c + e]);
+            for (int e2 = 0; e2 < 16; ++e2) {
+              float x0, x1;
+              f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[2 * e2]), __uint_as_float(sv[2 * e2 + 1])),
+                               SC, nl2[16 * c + e2]),
+                        x0, x1);
+              float p0, p1;
+              if ((e2 & 7) >= 5) {  // 3 of every 8 pairs on the FMA pipe, the rest on the SFU
+                p0 = exp2_poly<5>(x0);
+                p1 = exp2_poly<5>(x1);
+              } else {
+                p0 = fast_exp2(x0);
+                p1 = fast_exp2(x1);
+              }
+              A[e2 & 3] = f2_add(A[e2 & 3], f2_pack(p0, p1));
+            }
           }
         }
+        float a0, a1, a2, a3;
+        f2_unpack(f2_add(A[0], A[1]), a0, a1);
+        f2_unpack(f2_add(A[2], A[3]), a2, a3);
+        const float acc = (a0 + a1) + (a2 + a3);
         tc_fence_before();
         mbar_arrive(bar(kPBarFree + w));
         // add the two warpgroups' halves (exchange slot double-buffered by block
@@ -580,7 +672,14 @@ static cudaError_t launch_attn(const PrefillParams& p, bool gather, cudaStream_t
   a.out = p.out; a.lse = p.lse; a.status = p.status;
   const int ntile = p.G >= 2 ? 2 : 1;
   dim3 grid(n_tiles, p.Hq / ntile, p.B);
-  cudaError_t e;
+  // The kernel's setmaxnreg split assumes exactly kLaunchRegs registers per
+  // thread at launch; with fewer, the softmax warpgroups' increase could never
+  // be satisfied.  Refuse to launch a build that does not match.
+  cudaFuncAttributes fa;
+  cudaError_t e = gather ? cudaFuncGetAttributes(&fa, prefill_attn_kernel<true>)
+                         : cudaFuncGetAttributes(&fa, prefill_attn_kernel<false>);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs != kLaunchRegs) return cudaErrorNotSupported;
   if (gather) {
     e = cudaFuncSetAttribute(prefill_attn_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem);
     if (e != cudaSuccess) return e;

@@ -75,6 +75,16 @@ def test_null_and_misaligned_pointers(lib):
     assert lib.kascade_prefill_reuse(s, 256, P, P, P, P, P, 8, None, 0.1, P, P, P, ws, None) == INVALID
 
 
+def test_prefill_scale_must_be_positive(lib):
+    # the prefill kernels take the row maximum of the unscaled logits, which is
+    # the maximum of the scaled ones only for scale > 0
+    s = Shape(1, 32, 8, 128)
+    ws = 1 << 30
+    for bad in (0.0, -0.1, float("inf"), float("nan")):
+        assert lib.kascade_prefill_anchor(s, 256, P, P, P, bad, P, P, P, P, ws, None) == INVALID
+        assert lib.kascade_prefill_reuse(s, 256, P, P, P, P, P, 8, P, bad, P, P, P, ws, None) == INVALID
+
+
 def test_workspace_too_small(lib):
     s = Shape(4, 32, 8, 128)
     need = lib.kascade_decode_anchor_workspace_bytes(s, 32768)
