@@ -11,6 +11,8 @@
 //   degree 3: |rel err| < 1e-4      degree 5: |rel err| < 3e-7
 #pragma once
 
+#include "f32x2.cuh"
+
 namespace kascade {
 
 // coefficients of 2^f = sum_k c_k f^k, lowest order first
@@ -37,6 +39,30 @@ __device__ __forceinline__ float exp2_poly(float x) {
   }
   // n sits in the low bits of t (bias 0x4B400000); move it into the exponent
   return __int_as_float(__float_as_int(p) + ((__float_as_int(t) - 0x4B400000) << 23));
+}
+
+// exp2_poly<5> of two values on packed f32x2 arithmetic: the same operations
+// in the same order with the same roundings (t = x + M, n = t - M, f = x - n by
+// one fused multiply-add, Horner), so the results are bit-identical to the
+// scalar form.  The exponent add uses (t_bits << 23): the bias 0x4B400000
+// shifted left by 23 is 0 modulo 2^32.
+__device__ __forceinline__ void exp2_poly5_x2(float x0, float x1, float& y0, float& y1) {
+  constexpr float c0 = kExp2Deg5[0], c1 = kExp2Deg5[1], c2 = kExp2Deg5[2], c3 = kExp2Deg5[3],
+                  c4 = kExp2Deg5[4], c5 = kExp2Deg5[5];
+  const uint64_t X = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t T = f2_add(X, f2_pack(12582912.f, 12582912.f));
+  const uint64_t N = f2_add(T, f2_pack(-12582912.f, -12582912.f));
+  const uint64_t F = f2_fma(N, f2_pack(-1.f, -1.f), X);
+  uint64_t P = f2_fma(f2_pack(c5, c5), F, f2_pack(c4, c4));
+  P = f2_fma(P, F, f2_pack(c3, c3));
+  P = f2_fma(P, F, f2_pack(c2, c2));
+  P = f2_fma(P, F, f2_pack(c1, c1));
+  P = f2_fma(P, F, f2_pack(c0, c0));
+  float p0, p1, t0, t1;
+  f2_unpack(P, p0, p1);
+  f2_unpack(T, t0, t1);
+  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
 }
 
 }  // namespace kascade

@@ -75,7 +75,7 @@ constexpr uint32_t kAttnSmem = kAttnMisc + 256 + 1024;  // misc + alignment slac
 enum { kBarQ = 0, kBarKvFull = 1, kBarKvEmpty = 3, kBarS = 5, kBarP = 7, kBarO = 9, kAttnBars = 11 };
 
 // ---- pooling kernel layout ----
-constexpr int kPoolThreads = 384;
+constexpr int kPoolThreads = 384;  // warp 0 TMA, warp 1 MMA, warp 2 TMEM owner; warps 4-11 summing
 constexpr int kPoolHeads = 4;                           // query heads resident at once
 constexpr uint32_t kPoolQ = 0;
 constexpr uint32_t kPoolK = kPoolHeads * kTileBytes;    // 2 stages
@@ -83,8 +83,9 @@ constexpr uint32_t kPoolLse = kPoolK + 2 * kTileBytes;  // [kPoolHeads][128] flo
 constexpr uint32_t kPoolRed = kPoolLse + kPoolHeads * kTile * 4;  // [2][128] floats
 constexpr uint32_t kPoolMisc = kPoolRed + 2 * kTile * 4;
 constexpr uint32_t kPoolSmem = kPoolMisc + 256 + 1024;
-enum { kPBarQ = 0, kPBarKFull = 1, kPBarKEmpty = 3, kPBarS = 5, kPBarFree = 7, kPBarRedFull = 9,
-       kPBarRedEmpty = 11, kPoolBars = 13 };
+// per head of the round: S^T tile full (MMA commit) / free (read into registers, one arrival per warp)
+enum { kPBarQ = 0, kPBarKFull = 1, kPBarKEmpty = 3, kPBarS = 5, kPBarFree = 9, kPBarRedFull = 13,
+       kPBarRedEmpty = 15, kPoolBars = 17 };
 
 struct AttnArgs {
   int B, Hq, Hkv, G, N, n_tiles;
@@ -122,10 +123,6 @@ __device__ __forceinline__ constexpr uint64_t kmajor_step(int ks) {
   return (uint64_t)(((uint32_t)(ks >> 2) * kHalfBytes + (uint32_t)(ks & 3) * 32u) >> 4);
 }
 __device__ __forceinline__ constexpr uint64_t mnmajor_step(int ks) { return (uint64_t)(ks * 2048u >> 4); }
-
-__device__ __forceinline__ volatile int* abort_flag(uint8_t* smem, uint32_t misc) {
-  return reinterpret_cast<volatile int*>(smem + misc + 128);
-}
 
 template <bool GATHER>
 __global__ void __launch_bounds__(kAttnThreads, 1)
@@ -466,8 +463,8 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   float* lse2 = reinterpret_cast<float*>(smem + kPoolLse);
   float* red = reinterpret_cast<float*>(smem + kPoolRed);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kPoolMisc);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kPoolMisc + 96);
-  volatile int* s_abort = abort_flag(smem, kPoolMisc);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + kPoolMisc + 192);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kPoolMisc + 200);
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -479,8 +476,10 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   const int nblk = t;  // key blocks before the tile, per round
 
   if (tid == 0) {
-    for (int i = 0; i < kPoolBars; ++i)
-      mbar_init(bar(i), i >= kPBarFree ? 128u : 1u);
+    for (int i = 0; i < kPoolBars; ++i) {
+      const uint32_t count = i >= kPBarRedFull ? 128u : (i >= kPBarFree ? 4u : 1u);
+      mbar_init(bar(i), count);
+    }
     *s_abort = 0;
     mbar_fence_init();
   }
@@ -494,127 +493,151 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   const uint32_t tmem = *tmem_slot;
   float* prow = a.pooled + (((int64_t)b * a.n_tiles + t) * a.Hkv + h) * a.N;
   const float inv_count = 1.f / (float)(kTile * G);
-
-  for (int rd = 0; rd < n_rounds; ++rd) {
-    const int hg = min(kPoolHeads, G - rd * kPoolHeads);  // heads this round
-    const int gbase = h * G + rd * kPoolHeads;
-    // -lse of the round's heads (log2 domain), read in pairs by the summing warps
+  // -lse of a round's heads (log2 domain), read in pairs by the summing warps;
+  // every thread loads its share, then the CTA synchronises
+  auto load_lse2 = [&](int hg, int gbase) {
     for (int e = tid; e < hg * kTile; e += kPoolThreads) {
       const int j = e / kTile, q = e % kTile;
       lse2[e] = -a.lse[((int64_t)b * a.Hq + gbase + j) * a.N + (int64_t)kTile * t + q] * kLog2e;
     }
     __syncthreads();
-    const int it0 = rd * nblk;  // running block counter for stage / phase bookkeeping
-    if (warp == 0) {
-      // ---------------------------- TMA producer ----------------------------
-      if (lane == 0) {
-        mbar_expect_tx(bar(kPBarQ), hg * kTileBytes);
-        for (int j = 0; j < hg; ++j) {
-          const int y = (int)(((int64_t)b * a.Hq + gbase + j) * a.N + (int64_t)kTile * t);
-          tma_load_2d(sbase + kPoolQ + j * kTileBytes, &tm_q, 0, y, bar(kPBarQ));
-          tma_load_2d(sbase + kPoolQ + j * kTileBytes + kHalfBytes, &tm_q, 64, y, bar(kPBarQ));
+  };
+  // Each role runs its own copy of the round loop, so the compiler sizes every
+  // role's code for that role's register budget (setmaxnreg below).
+  if (warp < 4) {
+    setmaxnreg_dec<kOtherRegs>();
+    for (int rd = 0; rd < n_rounds; ++rd) {
+      const int hg = min(kPoolHeads, G - rd * kPoolHeads);  // heads this round
+      const int gbase = h * G + rd * kPoolHeads;
+      const int it0 = rd * nblk;  // running block counter for stage / phase bookkeeping
+      load_lse2(hg, gbase);
+      if (warp == 0) {
+        // ---------------------------- TMA producer ----------------------------
+        if (lane == 0) {
+          mbar_expect_tx(bar(kPBarQ), hg * kTileBytes);
+          for (int j = 0; j < hg; ++j) {
+            const int y = (int)(((int64_t)b * a.Hq + gbase + j) * a.N + (int64_t)kTile * t);
+            tma_load_2d(sbase + kPoolQ + j * kTileBytes, &tm_q, 0, y, bar(kPBarQ));
+            tma_load_2d(sbase + kPoolQ + j * kTileBytes + kHalfBytes, &tm_q, 64, y, bar(kPBarQ));
+          }
+          for (int jb = 0; jb < nblk; ++jb) {
+            const int it = it0 + jb, st = it & 1;
+            if (it >= 2 && !mbar_wait(bar(kPBarKEmpty + st), ((it >> 1) - 1) & 1, a.status)) { *s_abort = 1; break; }
+            if (*s_abort) break;
+            const uint32_t ks = sbase + kPoolK + st * kTileBytes;
+            mbar_expect_tx(bar(kPBarKFull + st), kTileBytes);
+            tma_load_2d(ks, &tm_k, 0, kv_row0 + kTile * jb, bar(kPBarKFull + st));
+            tma_load_2d(ks + kHalfBytes, &tm_k, 64, kv_row0 + kTile * jb, bar(kPBarKFull + st));
+          }
         }
-        for (int jb = 0; jb < nblk; ++jb) {
-          const int it = it0 + jb, st = it & 1;
-          if (it >= 2 && !mbar_wait(bar(kPBarKEmpty + st), ((it >> 1) - 1) & 1, a.status)) { *s_abort = 1; break; }
-          if (*s_abort) break;
-          const uint32_t ks = sbase + kPoolK + st * kTileBytes;
-          mbar_expect_tx(bar(kPBarKFull + st), kTileBytes);
-          tma_load_2d(ks, &tm_k, 0, kv_row0 + kTile * jb, bar(kPBarKFull + st));
-          tma_load_2d(ks + kHalfBytes, &tm_k, 64, kv_row0 + kTile * jb, bar(kPBarKFull + st));
-        }
-      }
-    } else if (warp == 1) {
-      // ---------------------------- MMA issuer ------------------------------
-      if (lane == 0) {
-        const uint32_t idesc = idesc_bf16(128, 128, false, false);
-        bool ok = mbar_wait(bar(kPBarQ), rd & 1, a.status);
-        for (int jb = 0; ok && jb < nblk; ++jb) {
-          const int it = it0 + jb, st = it & 1;
-          if (!(ok = mbar_wait(bar(kPBarKFull + st), (it >> 1) & 1, a.status))) break;
-          const uint64_t dk = kmajor_desc(sbase + kPoolK + st * kTileBytes, 0);
-          for (int w = 0; w < 2; ++w) {
-            // region w holds heads 2w, 2w+1 of the round; wait until its summing
-            // warpgroup has read the previous block
-            if (it >= 1 && !(ok = mbar_spin(bar(kPBarFree + w), (it - 1) & 1, a.status))) break;
-            tc_fence_after();
-            for (int jj = 2 * w; jj < min(2 * w + 2, hg); ++jj) {
-              const uint64_t dq = kmajor_desc(sbase + kPoolQ + jj * kTileBytes, 0);
+      } else if (warp == 1) {
+        // ---------------------------- MMA issuer ------------------------------
+        // S^T_g = K Q_g^T for each head g of the round into its own 128 TMEM
+        // columns, as soon as the summing warps have read that head's previous tile.
+        if (lane == 0) {
+          const uint32_t idesc = idesc_bf16(128, 128, false, false);
+          bool ok = mbar_wait(bar(kPBarQ), rd & 1, a.status);
+          for (int jb = 0; ok && jb < nblk; ++jb) {
+            const int it = it0 + jb, st = it & 1;
+            if (!(ok = mbar_wait(bar(kPBarKFull + st), (it >> 1) & 1, a.status))) break;
+            const uint64_t dk = kmajor_desc(sbase + kPoolK + st * kTileBytes, 0);
+            for (int g = 0; g < hg; ++g) {
+              if (it >= 1 && !(ok = mbar_spin(bar(kPBarFree + g), (it - 1) & 1, a.status))) break;
+              tc_fence_after();
+              const uint64_t dq = kmajor_desc(sbase + kPoolQ + g * kTileBytes, 0);
 #pragma unroll
               for (int k16 = 0; k16 < 8; ++k16)
-                umma_ss(tmem + 128 * jj, dk + kmajor_step(k16), dq + kmajor_step(k16), idesc,
-                        k16 > 0 ? 1u : 0u);
+                umma_ss(tmem + 128 * g, dk + kmajor_step(k16), dq + kmajor_step(k16), idesc, k16 > 0 ? 1u : 0u);
+              umma_commit(bar(kPBarS + g));
             }
-            umma_commit(bar(kPBarS + w));
+            if (!ok) break;
+            umma_commit(bar(kPBarKEmpty + st));
+            if (*s_abort) { ok = false; break; }
           }
-          if (!ok) break;
-          umma_commit(bar(kPBarKEmpty + st));
-          if (*s_abort) { ok = false; break; }
+          if (!ok) *s_abort = 1;
         }
-        if (!ok) *s_abort = 1;
       }
-    } else if (warp >= 4) {
-      // ------------------- summing warpgroups (heads 2w, 2w+1) ---------------
-      const int w = (warp - 4) >> 2;
-      const int key = tid - 128 - 128 * w;  // TMEM lane
-      const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-      for (int jb = 0; jb < nblk; ++jb) {
-        const int it = it0 + jb;
-        if (!mbar_wait(bar(kPBarS + w), it & 1, a.status) || *s_abort) { *s_abort = 1; break; }
-        tc_fence_after();
-        // sum over the queries of exp2(s * sc - lse2), two per packed instruction
-        uint64_t A[4] = {0ull, 0ull, 0ull, 0ull};
+      __syncthreads();  // round done: Q tiles and lse2 may be replaced
+    }
+  } else {
+    setmaxnreg_inc<kSoftmaxRegs>();
+    for (int rd = 0; rd < n_rounds; ++rd) {
+      const int hg = min(kPoolHeads, G - rd * kPoolHeads);
+      const int gbase = h * G + rd * kPoolHeads;
+      const int it0 = rd * nblk;
+      load_lse2(hg, gbase);
+      {
+        // ------------------- summing warpgroups (heads w, w + 2) ---------------
+        // Thread = key (TMEM lane).  A head's 128 scores are read into registers
+        // and its tile released to the MMA before the exponentials are summed.
+        const int w = (warp >> 2) - 1;
+        const int key = (warp & 3) * 32 + lane;
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const uint64_t SC = f2_pack(a.scale_log2, a.scale_log2);
-        for (int jj = 2 * w; jj < min(2 * w + 2, hg); ++jj) {
-          const uint64_t* nl2 = reinterpret_cast<const uint64_t*>(lse2 + jj * kTile);
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t sv[32];
-            tmem_ld32(tmem + 128 * jj + lane_base + 32 * c, sv);
+        for (int jb = 0; jb < nblk; ++jb) {
+          const int it = it0 + jb;
+          uint64_t A[4] = {0ull, 0ull, 0ull, 0ull};
+          bool ok = true;
+          for (int g = w; g < hg; g += 2) {
+            if (!(ok = mbar_wait(bar(kPBarS + g), it & 1, a.status)) || *s_abort) { ok = false; break; }
+            tc_fence_after();
+            uint32_t v[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32(tmem + 128 * g + lane_base + 32 * c, v[c]);
             tmem_wait_ld();
 #pragma unroll
-            for (int e2 = 0; e2 < 16; ++e2) {
-              float x0, x1;
-              f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[2 * e2]), __uint_as_float(sv[2 * e2 + 1])),
-                               SC, nl2[16 * c + e2]),
-                        x0, x1);
-              float p0, p1;
-              if ((e2 & 7) >= 5) {  // 3 of every 8 pairs on the FMA pipe, the rest on the SFU
-                p0 = exp2_poly<5>(x0);
-                p1 = exp2_poly<5>(x1);
-              } else {
-                p0 = fast_exp2(x0);
-                p1 = fast_exp2(x1);
+            for (int c = 0; c < 4; ++c) reg_fence32(v[c]);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kPBarFree + g));
+            // sum over the queries of exp2(s * sc - lse2), two per packed instruction;
+            // 3 of every 8 pairs on the FMA pipe, the rest on the SFU
+            const uint64_t* nl2 = reinterpret_cast<const uint64_t*>(lse2 + g * kTile);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              asm volatile("" ::: "memory");  // keep each chunk's lse loads next to their use
+#pragma unroll
+              for (int e2 = 0; e2 < 16; ++e2) {
+                float x0, x1;
+                f2_unpack(f2_fma(f2_pack(__uint_as_float(v[c][2 * e2]), __uint_as_float(v[c][2 * e2 + 1])),
+                                 SC, nl2[16 * c + e2]),
+                          x0, x1);
+                float p0, p1;
+                if ((e2 & 7) >= 5) {
+                  exp2_poly5_x2(x0, x1, p0, p1);
+                } else {
+                  p0 = fast_exp2(x0);
+                  p1 = fast_exp2(x1);
+                }
+                A[e2 & 3] = f2_add(A[e2 & 3], f2_pack(p0, p1));
               }
-              A[e2 & 3] = f2_add(A[e2 & 3], f2_pack(p0, p1));
             }
           }
-        }
-        float a0, a1, a2, a3;
-        f2_unpack(f2_add(A[0], A[1]), a0, a1);
-        f2_unpack(f2_add(A[2], A[3]), a2, a3);
-        const float acc = (a0 + a1) + (a2 + a3);
-        tc_fence_before();
-        mbar_arrive(bar(kPBarFree + w));
-        // add the two warpgroups' halves (exchange slot double-buffered by block
-        // parity, guarded by bounded mbarrier waits) and write the pooled value
-        const int sl = it & 1;
-        float* slot = red + sl * kTile;
-        if (w == 1) {
-          if (it >= 2 && !mbar_wait(bar(kPBarRedEmpty + sl), ((it >> 1) - 1) & 1, a.status)) { *s_abort = 1; break; }
-          slot[key] = acc;
-          mbar_arrive(bar(kPBarRedFull + sl));
-        } else {
-          if (!mbar_wait(bar(kPBarRedFull + sl), (it >> 1) & 1, a.status)) { *s_abort = 1; break; }
-          const float tot = acc + slot[key];
-          mbar_arrive(bar(kPBarRedEmpty + sl));
-          const int col = kTile * jb + key;
-          if (rd == 0) prow[col] = tot * inv_count;
-          else prow[col] += tot * inv_count;
+          if (!ok) { *s_abort = 1; break; }
+          float a0, a1, a2, a3;
+          f2_unpack(f2_add(A[0], A[1]), a0, a1);
+          f2_unpack(f2_add(A[2], A[3]), a2, a3);
+          const float acc = (a0 + a1) + (a2 + a3);
+          // add the two warpgroups' halves (exchange slot double-buffered by block
+          // parity, guarded by bounded mbarrier waits) and write the pooled value
+          const int sl = it & 1;
+          float* slot = red + sl * kTile;
+          if (w == 1) {
+            if (it >= 2 && !mbar_wait(bar(kPBarRedEmpty + sl), ((it >> 1) - 1) & 1, a.status)) { *s_abort = 1; break; }
+            slot[key] = acc;
+            mbar_arrive(bar(kPBarRedFull + sl));
+          } else {
+            if (!mbar_wait(bar(kPBarRedFull + sl), (it >> 1) & 1, a.status)) { *s_abort = 1; break; }
+            const float tot = acc + slot[key];
+            mbar_arrive(bar(kPBarRedEmpty + sl));
+            const int col = kTile * jb + key;
+            if (rd == 0) prow[col] = tot * inv_count;
+            else prow[col] += tot * inv_count;
+          }
         }
       }
+      __syncthreads();
     }
-    __syncthreads();  // round done: Q tiles and lse2 may be replaced
   }
   tc_fence_before();
   __syncthreads();
@@ -705,6 +728,10 @@ cudaError_t launch_prefill_anchor(const PrefillParams& p, cudaStream_t st) {
   a.B = p.B; a.Hq = p.Hq; a.Hkv = p.Hkv; a.G = p.G; a.N = p.N; a.n_tiles = n_tiles;
   a.scale_log2 = (float)((double)p.scale * 1.4426950408889634);
   a.lse = p.lse; a.pooled = p.pooled; a.status = p.status;
+  cudaFuncAttributes fa;  // same setmaxnreg split as the attention kernel
+  e = cudaFuncGetAttributes(&fa, prefill_pool_kernel);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs != kLaunchRegs) return cudaErrorNotSupported;
   e = cudaFuncSetAttribute(prefill_pool_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPoolSmem);
   if (e != cudaSuccess) return e;
   dim3 grid(n_tiles - 1, p.Hkv, p.B);
