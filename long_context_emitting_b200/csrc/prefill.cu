@@ -477,7 +477,7 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
   if (tid == 0) {
     for (int i = 0; i < kPoolBars; ++i) {
-      const uint32_t count = i >= kPBarRedFull ? 128u : (i >= kPBarFree ? 4u : 1u);
+      const uint32_t count = i >= kPBarFree ? 4u : 1u;  // free / exchange: one arrival per warp
       mbar_init(bar(i), count);
     }
     *s_abort = 0;
@@ -625,11 +625,13 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           if (w == 1) {
             if (it >= 2 && !mbar_wait(bar(kPBarRedEmpty + sl), ((it >> 1) - 1) & 1, a.status)) { *s_abort = 1; break; }
             slot[key] = acc;
-            mbar_arrive(bar(kPBarRedFull + sl));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kPBarRedFull + sl));
           } else {
             if (!mbar_wait(bar(kPBarRedFull + sl), (it >> 1) & 1, a.status)) { *s_abort = 1; break; }
             const float tot = acc + slot[key];
-            mbar_arrive(bar(kPBarRedEmpty + sl));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kPBarRedEmpty + sl));
             const int col = kTile * jb + key;
             if (rd == 0) prow[col] = tot * inv_count;
             else prow[col] += tot * inv_count;
