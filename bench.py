@@ -433,18 +433,36 @@ def main():
     if api.device_status() != 0:
         raise RuntimeError("device status set during warm-up")
 
-    # Each schedule step (all layers) is captured once as a CUDA graph, with
-    # event-record nodes around every op; the timed region replays the graphs.
+    # Each schedule step (all layers) is captured once as a CUDA graph with an
+    # event-record node at each end; the timed region replays these graphs.
+    # A second capture of each step carries event nodes around every op; it is
+    # replayed after the timed region for the per-op breakdown, so the timed
+    # steps contain no extra nodes between kernels.
     from long_context_emitting_b200.schedule import StepGraph
 
     rt = _Cudart()
     timer = GraphOpTimer(rt)
+    spans = {}
     capturing = torch.cuda.is_current_stream_capturing
-    gdec = StepGraph(lambda: decode_step(dec[1], dec[2], dec[3], dec[4],
-                                         timer if capturing() else None)) if dec else None
-    dec_marks = len(timer.marks)
-    gpre = StepGraph(lambda: prefill_step(pre[1], pre[2], pre[3], pre[4],
-                                          timer if capturing() else None)) if pre else None
+
+    def spanned(name, fn):
+        def run():
+            if not capturing():
+                fn()
+                return
+            s, e = rt.create(), rt.create()
+            rt.record_external(s)
+            fn()
+            rt.record_external(e)
+            spans[name] = (s, e)
+        return run
+
+    gdec = StepGraph(spanned("dec", lambda: decode_step(dec[1], dec[2], dec[3], dec[4]))) if dec else None
+    gpre = StepGraph(spanned("pre", lambda: prefill_step(pre[1], pre[2], pre[3], pre[4]))) if pre else None
+    gdec_ops = StepGraph(lambda: decode_step(dec[1], dec[2], dec[3], dec[4],
+                                             timer if capturing() else None)) if dec else None
+    gpre_ops = StepGraph(lambda: prefill_step(pre[1], pre[2], pre[3], pre[4],
+                                              timer if capturing() else None)) if pre else None
     if api.device_status() != 0:
         raise RuntimeError("device status set during capture")
 
@@ -460,9 +478,8 @@ def main():
         if gpre:
             gpre.replay()
         torch.cuda.synchronize()
-        timer.collect()
-        d = rt.elapsed_ms(timer.marks[0][1], timer.marks[dec_marks - 1][2]) if gdec else 0.0
-        p = rt.elapsed_ms(timer.marks[dec_marks][1], timer.marks[-1][2]) if gpre else 0.0
+        d = rt.elapsed_ms(*spans["dec"]) if gdec else 0.0
+        p = rt.elapsed_ms(*spans["pre"]) if gpre else 0.0
         dec_ms_steps.append(d)
         pre_ms_steps.append(p)
         step_ms.append(d + p)
@@ -471,6 +488,14 @@ def main():
     clk = clocks.stop()
     if api.device_status() != 0:
         raise RuntimeError("device status set during the timed steps")
+    # per-op breakdown (outside the timed region)
+    for _ in range(min(args.steps, 10)):
+        if gdec_ops:
+            gdec_ops.replay()
+        if gpre_ops:
+            gpre_ops.replay()
+        torch.cuda.synchronize()
+        timer.collect()
     ms_per_step = dist.max(sum(step_ms) / args.steps)
     N = dist.world
 

@@ -98,28 +98,15 @@ struct Blk {
   bool oka, okb;     // rows present
 };
 
-template <bool GATHER>
-__device__ __forceinline__ void load_blk(Blk& x, int i0, int i_end, const int32_t* rows, int T,
-                                         const uint16_t* Kb, const uint16_t* Vb, int gid, int tig,
-                                         unsigned* status) {
+// Loads one 16-row block of the anchor's contiguous K/V stream into registers.
+__device__ __forceinline__ void load_blk(Blk& x, int i0, int i_end, const uint16_t* Kb, const uint16_t* Vb,
+                                         int gid, int tig) {
   x.ia = i0 + gid;
   x.ib = i0 + gid + 8;
   x.oka = x.ia < i_end;
   x.okb = x.ib < i_end;
-  int ra = x.ia, rb = x.ib;
-  if (GATHER) {
-    ra = x.oka ? __ldg(rows + x.ia) : 0;
-    rb = x.okb ? __ldg(rows + x.ib) : 0;
-    if (x.oka && (ra < 0 || ra >= T)) { flag_status(status, kStatusBadIndex); x.oka = false; }
-    if (x.okb && (rb < 0 || rb >= T)) { flag_status(status, kStatusBadIndex); x.okb = false; }
-    // masked lanes address row 0 (T >= 1 here), so no address leaves the sequence
-    if (!x.oka) ra = 0;
-    if (!x.okb) rb = 0;
-  } else {
-    // masked lanes address the block's first row, which is < i_end <= T
-    if (!x.oka) ra = i0;
-    if (!x.okb) rb = i0;
-  }
+  // masked lanes address the block's first row, which is < i_end <= T
+  const int ra = x.oka ? x.ia : i0, rb = x.okb ? x.ib : i0;
   const uint16_t* kpa = Kb + (int64_t)ra * kHeadDim + 8 * tig;
   const uint16_t* kpb = Kb + (int64_t)rb * kHeadDim + 8 * tig;
   const uint16_t* vpa = Vb + (int64_t)ra * kHeadDim + 8 * tig;
@@ -204,12 +191,9 @@ __device__ __forceinline__ void compute_blk(const Blk& x, WarpState& w, const ui
   }
 }
 
-// Anchor (contiguous stream): two register buffers, the next block's loads in
-// flight during the current block's math, 2 CTAs per SM.  Reuse (gather): one
-// buffer and 4 CTAs per SM, since more resident warps hide the scattered-row
-// latency better than deeper per-warp pipelining.
-template <bool GATHER>
-__global__ void __launch_bounds__(kThreads, GATHER ? 4 : 2) decode_split_kernel(const SplitArgs a) {
+// Decode anchor over the contiguous K/V stream: two register buffers (the
+// next block's loads in flight during the current block's math), 2 CTAs per SM.
+__global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const SplitArgs a) {
   __shared__ float sm_o[kWarps][8][kHeadDim];
   __shared__ float sm_m[kWarps][8];
   __shared__ float sm_l[kWarps][8];
@@ -222,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, GATHER ? 4 : 2) decode_split_kernel(
   int T;
   int64_t off;
   const int32_t* rows;
-  int n_items = resolve_rows<GATHER>(a, b, h, T, off, rows);
+  int n_items = resolve_rows<false>(a, b, h, T, off, rows);
   if (n_items < 0) {
     if (threadIdx.x == 0 && split == 0) flag_status(a.status, kStatusBadIndex);
     n_items = 0;
@@ -250,28 +234,17 @@ __global__ void __launch_bounds__(kThreads, GATHER ? 4 : 2) decode_split_kernel(
 #pragma unroll
   for (int i = 0; i < 8; ++i) ws.o[i][0] = ws.o[i][1] = ws.o[i][2] = ws.o[i][3] = 0.f;
 
-  float* lrow = nullptr;
-  if (!GATHER) lrow = a.logits + ((int64_t)b * a.Hkv + h) * a.max_T * G;
+  float* lrow = a.logits + ((int64_t)b * a.Hkv + h) * a.max_T * G;
 
-  // Two register buffers: the next block's loads are in flight while the
-  // current block is computed.
-  if (!GATHER) {
   Blk x0, x1;
-  if (i_begin < i_end) load_blk<GATHER>(x0, i_begin, i_end, rows, T, Kb, Vb, gid, tig, a.status);
+  if (i_begin < i_end) load_blk(x0, i_begin, i_end, Kb, Vb, gid, tig);
   for (int i0 = i_begin; i0 < i_end; i0 += 32) {
     const bool has1 = i0 + 16 < i_end;
-    if (has1) load_blk<GATHER>(x1, i0 + 16, i_end, rows, T, Kb, Vb, gid, tig, a.status);
-    compute_blk<GATHER>(x0, ws, qf, a.scale_log2, lrow, G, tig);
+    if (has1) load_blk(x1, i0 + 16, i_end, Kb, Vb, gid, tig);
+    compute_blk<false>(x0, ws, qf, a.scale_log2, lrow, G, tig);
     if (!has1) break;
-    if (i0 + 32 < i_end) load_blk<GATHER>(x0, i0 + 32, i_end, rows, T, Kb, Vb, gid, tig, a.status);
-    compute_blk<GATHER>(x1, ws, qf, a.scale_log2, lrow, G, tig);
-  }
-  } else {
-  for (int i0 = i_begin; i0 < i_end; i0 += 16) {
-    Blk x0;
-    load_blk<GATHER>(x0, i0, i_end, rows, T, Kb, Vb, gid, tig, a.status);
-    compute_blk<GATHER>(x0, ws, qf, a.scale_log2, lrow, G, tig);
-  }
+    if (i0 + 32 < i_end) load_blk(x0, i0 + 32, i_end, Kb, Vb, gid, tig);
+    compute_blk<false>(x1, ws, qf, a.scale_log2, lrow, G, tig);
   }
 
   // ---- merge the 4 warps of the CTA --------------------------------------
@@ -712,7 +685,7 @@ static cudaError_t launch_decode(const DecodeParams& p, bool gather, cudaStream_
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }
-  decode_split_kernel<false><<<grid, kThreads, 0, st>>>(a);
+  decode_split_kernel<<<grid, kThreads, 0, st>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
