@@ -22,7 +22,10 @@
 //                 at once, so the row maximum needs no exchange between
 //                 threads.  Online softmax in base 2 (the running maximum is
 //                 raised only when a block exceeds it by 2^8, so O is rarely
-//                 rescaled); P goes back to TMEM as bf16 over the row's S.
+//                 rescaled); P goes back to TMEM as bf16 over the row's S, in
+//                 two halves of 64 keys, each handed to the MMA as soon as it
+//                 is stored (PV of the first half overlaps the exponentials of
+//                 the second).
 //   The MMA thread alternates between the tiles, so the tensor cores work on
 //   one tile while the other tile's softmax runs.  The softmax warpgroups take
 //   registers from the third one (setmaxnreg; the launch checks the split).
@@ -31,12 +34,14 @@
 // prefill_pool_kernel
 //   One CTA per (tile t >= 1, KV head, sequence).  For each key block before
 //   the tile it computes S^T = K Q_g^T for the group's query heads (keys on
-//   TMEM lanes, queries on columns), so a thread owns one key and sums
-//   exp2(s - lse2) over the tile's queries in registers (3 of 8 exponentials
-//   on the FMA pipe, the rest on the SFU).  Warp roles: a TMA
-//   producer, an MMA issuer and two warpgroups that each sum half of the heads
-//   (ping-ponging on two TMEM regions); the two halves are added through shared
-//   memory and pooled = sum / (128 G) is written once, without atomics.
+//   TMEM lanes, queries on columns, one 128-column TMEM tile per head), so a
+//   thread owns one key and sums exp2(s - lse2) over the tile's queries in
+//   registers (3 of 8 exponentials on the FMA pipe, the rest on the SFU).
+//   Warp roles (640 threads): a TMA producer and an MMA issuer in warpgroup 0,
+//   and four summing warpgroups, one per head of the round; a head's tile goes
+//   back to the MMA as soon as its scores are in registers.  The heads' sums
+//   are added through shared memory and pooled = sum / (128 G) is written
+//   once, without atomics.
 #include "exp2_poly.cuh"
 #include "f32x2.cuh"
 #include "tcgen05.cuh"
@@ -72,18 +77,26 @@ constexpr uint32_t kAttnQ = 0;                         // 2 query tiles
 constexpr uint32_t kAttnKV = 2 * kTileBytes;           // stage s: K at +2s*tile, V at +(2s+1)*tile
 constexpr uint32_t kAttnMisc = kAttnKV + 4 * kTileBytes;
 constexpr uint32_t kAttnSmem = kAttnMisc + 256 + 1024;  // misc + alignment slack
-enum { kBarQ = 0, kBarKvFull = 1, kBarKvEmpty = 3, kBarS = 5, kBarP = 7, kBarO = 9, kAttnBars = 11 };
+enum { kBarQ = 0, kBarKvFull = 1, kBarKvEmpty = 3, kBarS = 5, kBarP = 7, kBarO = 11, kAttnBars = 13 };
 
 // ---- pooling kernel layout ----
-constexpr int kPoolThreads = 384;  // warp 0 TMA, warp 1 MMA, warp 2 TMEM owner; warps 4-11 summing
+constexpr int kPoolThreads = 640;  // warpgroup 0: TMA (warp 0), MMA (warp 1), TMEM owner (warp 2);
+                                   // warpgroups 1-4: summing, one per head of the round
 constexpr int kPoolHeads = 4;                           // query heads resident at once
+// setmaxnreg split of the 96 x 640 launch registers: warpgroup 0 releases down to
+// 64, the four summing warpgroups take exactly that.
+constexpr int kPoolLaunchRegs = 96, kPoolSumRegs = 104, kPoolCtlRegs = 64;
+static_assert((kPoolLaunchRegs - kPoolCtlRegs) * 128 >= (kPoolSumRegs - kPoolLaunchRegs) * 512,
+              "summing register increase must fit in what warpgroup 0 releases");
+static_assert(kPoolLaunchRegs * kPoolThreads <= 65536, "launch registers exceed the SM");
 constexpr uint32_t kPoolQ = 0;
 constexpr uint32_t kPoolK = kPoolHeads * kTileBytes;    // 2 stages
 constexpr uint32_t kPoolLse = kPoolK + 2 * kTileBytes;  // [kPoolHeads][128] floats
-constexpr uint32_t kPoolRed = kPoolLse + kPoolHeads * kTile * 4;  // [2][128] floats
-constexpr uint32_t kPoolMisc = kPoolRed + 2 * kTile * 4;
+constexpr uint32_t kPoolRed = kPoolLse + kPoolHeads * kTile * 4;  // [2 slots][3 heads][128] floats
+constexpr uint32_t kPoolMisc = kPoolRed + 2 * 3 * kTile * 4;
 constexpr uint32_t kPoolSmem = kPoolMisc + 256 + 1024;
-// per head of the round: S^T tile full (MMA commit) / free (read into registers, one arrival per warp)
+// per head of the round: S^T tile full (MMA commit) / free (read into registers,
+// one arrival per warp); partial-sum exchange: heads 1-3 -> head 0's warpgroup
 enum { kPBarQ = 0, kPBarKFull = 1, kPBarKEmpty = 3, kPBarS = 5, kPBarFree = 9, kPBarRedFull = 13,
        kPBarRedEmpty = 15, kPoolBars = 17 };
 
@@ -169,7 +182,7 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
   if (tid == 0) {
     for (int i = 0; i < kAttnBars; ++i) {
-      const bool per_warp = i >= kBarP && i < kBarP + 2;  // 4 softmax warps per tile
+      const bool per_warp = i >= kBarP && i < kBarP + 4;  // 4 softmax warps per tile
       mbar_init(bar(i), per_warp ? 4u : 1u);
     }
     *s_abort = 0;
@@ -269,11 +282,11 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             umma_ss(d, dq + kmajor_step(k16), dk + kmajor_step(k16), idesc_s, k16 > 0 ? 1u : 0u);
         };
         // P (128 keys as bf16 pairs) sits in columns 0..63 of the tile's S region.
-        auto issue_pv = [&](int i, int st, bool acc) {
+        auto issue_pv = [&](int i, int st, bool acc, int k0) {  // keys 16*k0 .. 16*k0+63
           const uint64_t dv = st ? dv1 : dv0;
           const uint32_t d = tmem + 256 * i + 128, pa = tmem + 256 * i;
 #pragma unroll
-          for (int k16 = 0; k16 < 8; ++k16)
+          for (int k16 = k0; k16 < k0 + 4; ++k16)
             umma_ts(d, pa + 8 * k16, dv + mnmajor_step(k16), idesc_o, (acc || k16 > 0) ? 1u : 0u);
         };
         bool ok = mbar_wait(bar(kBarQ), 0, a.status);
@@ -291,7 +304,10 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           // tile 0: PV of this block, then S of the next block
           if (!(ok = mbar_spin(bar(kBarP + 0), j & 1, a.status))) break;
           tc_fence_after();
-          issue_pv(0, st, j > 0);
+          issue_pv(0, st, j > 0, 0);
+          if (!(ok = mbar_spin(bar(kBarP + 1), j & 1, a.status))) break;
+          tc_fence_after();
+          issue_pv(0, st, j > 0, 4);
           if (more) {
             if (!(ok = mbar_wait(bar(kBarKvFull + (st ^ 1)), ((j + 1) >> 1) & 1, a.status))) break;
             tc_fence_after();
@@ -299,9 +315,12 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             umma_commit(bar(kBarS + 0));
           }
           if (ntile == 2) {
-            if (!(ok = mbar_spin(bar(kBarP + 1), j & 1, a.status))) break;
+            if (!(ok = mbar_spin(bar(kBarP + 2), j & 1, a.status))) break;
             tc_fence_after();
-            issue_pv(1, st, j > 0);
+            issue_pv(1, st, j > 0, 0);
+            if (!(ok = mbar_spin(bar(kBarP + 3), j & 1, a.status))) break;
+            tc_fence_after();
+            issue_pv(1, st, j > 0, 4);
           }
           umma_commit(bar(kBarKvEmpty + st));  // K/V stage free once these MMAs complete
           if (ntile == 2 && more) {
@@ -408,6 +427,13 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             L[e2 & 3] = f2_add(L[e2 & 3], f2_pack(p0, p1));
             pw[e2] = pack_bf16x2(p0, p1);
           }
+          if (c == 2) {
+            // keys 0..63 are stored: hand them to the MMA before the rest
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kBarP + 2 * i));
+          }
           tmem_st16(tS + 16 * c, pw);
         }
         float l0, l1, l2, l3;
@@ -417,7 +443,7 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(kBarP + i));  // one arrival per warp, 4 per tile
+        if (lane == 0) mbar_arrive(bar(kBarP + 2 * i + 1));  // one arrival per warp, 4 per tile
       }
       if (!ok) *s_abort = 1;
       // ---- epilogue: O / l --------------------------------------------------------
@@ -463,8 +489,8 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   float* lse2 = reinterpret_cast<float*>(smem + kPoolLse);
   float* red = reinterpret_cast<float*>(smem + kPoolRed);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kPoolMisc);
-  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + kPoolMisc + 192);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kPoolMisc + 200);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + kPoolMisc + 224);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kPoolMisc + 232);
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -477,7 +503,8 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
   if (tid == 0) {
     for (int i = 0; i < kPoolBars; ++i) {
-      const uint32_t count = i >= kPBarFree ? 4u : 1u;  // free / exchange: one arrival per warp
+      // free: the head's 4 warps; exchange full: 12 warps of heads 1-3; empty: head 0's 4 warps
+      const uint32_t count = (i >= kPBarRedFull && i < kPBarRedEmpty) ? 12u : (i >= kPBarFree ? 4u : 1u);
       mbar_init(bar(i), count);
     }
     *s_abort = 0;
@@ -505,7 +532,7 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   // Each role runs its own copy of the round loop, so the compiler sizes every
   // role's code for that role's register budget (setmaxnreg below).
   if (warp < 4) {
-    setmaxnreg_dec<kOtherRegs>();
+    setmaxnreg_dec<kPoolCtlRegs>();
     for (int rd = 0; rd < n_rounds; ++rd) {
       const int hg = min(kPoolHeads, G - rd * kPoolHeads);  // heads this round
       const int gbase = h * G + rd * kPoolHeads;
@@ -560,82 +587,92 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       __syncthreads();  // round done: Q tiles and lse2 may be replaced
     }
   } else {
-    setmaxnreg_inc<kSoftmaxRegs>();
+    setmaxnreg_inc<kPoolSumRegs>();
+    // ------------------- summing warpgroups (one head each) -------------------
+    // Thread = key (TMEM lane).  The head's 128 scores are read in two halves
+    // of 64 queries; the tile is released to the MMA once the second half is in
+    // registers, before its exponentials are summed.
+    const int g = (warp >> 2) - 1;  // head of the round handled by this warpgroup
+    const int key = (warp & 3) * 32 + lane;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint64_t SC = f2_pack(a.scale_log2, a.scale_log2);
     for (int rd = 0; rd < n_rounds; ++rd) {
       const int hg = min(kPoolHeads, G - rd * kPoolHeads);
       const int gbase = h * G + rd * kPoolHeads;
       const int it0 = rd * nblk;
       load_lse2(hg, gbase);
-      {
-        // ------------------- summing warpgroups (heads w, w + 2) ---------------
-        // Thread = key (TMEM lane).  A head's 128 scores are read into registers
-        // and its tile released to the MMA before the exponentials are summed.
-        const int w = (warp >> 2) - 1;
-        const int key = (warp & 3) * 32 + lane;
-        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        const uint64_t SC = f2_pack(a.scale_log2, a.scale_log2);
-        for (int jb = 0; jb < nblk; ++jb) {
-          const int it = it0 + jb;
-          uint64_t A[4] = {0ull, 0ull, 0ull, 0ull};
-          bool ok = true;
-          for (int g = w; g < hg; g += 2) {
-            if (!(ok = mbar_wait(bar(kPBarS + g), it & 1, a.status)) || *s_abort) { ok = false; break; }
-            tc_fence_after();
-            uint32_t v[4][32];
+      for (int jb = 0; jb < nblk; ++jb) {
+        const int it = it0 + jb;
+        uint64_t A[4] = {0ull, 0ull, 0ull, 0ull};
+        // sum over 64 queries of exp2(s * sc - lse2), two per packed instruction;
+        // 3 of every 8 pairs on the FMA pipe, the rest on the SFU
+        auto sum_half = [&](const uint32_t (&v)[2][32], int q0) {
+          const uint64_t* nl2 = reinterpret_cast<const uint64_t*>(lse2 + g * kTile + q0);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(tmem + 128 * g + lane_base + 32 * c, v[c]);
-            tmem_wait_ld();
+          for (int c = 0; c < 2; ++c) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) reg_fence32(v[c]);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(kPBarFree + g));
-            // sum over the queries of exp2(s * sc - lse2), two per packed instruction;
-            // 3 of every 8 pairs on the FMA pipe, the rest on the SFU
-            const uint64_t* nl2 = reinterpret_cast<const uint64_t*>(lse2 + g * kTile);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              asm volatile("" ::: "memory");  // keep each chunk's lse loads next to their use
-#pragma unroll
-              for (int e2 = 0; e2 < 16; ++e2) {
-                float x0, x1;
-                f2_unpack(f2_fma(f2_pack(__uint_as_float(v[c][2 * e2]), __uint_as_float(v[c][2 * e2 + 1])),
-                                 SC, nl2[16 * c + e2]),
-                          x0, x1);
-                float p0, p1;
-                if ((e2 & 7) >= 5) {
-                  exp2_poly5_x2(x0, x1, p0, p1);
-                } else {
-                  p0 = fast_exp2(x0);
-                  p1 = fast_exp2(x1);
-                }
-                A[e2 & 3] = f2_add(A[e2 & 3], f2_pack(p0, p1));
+            for (int e2 = 0; e2 < 16; ++e2) {
+              float x0, x1;
+              f2_unpack(f2_fma(f2_pack(__uint_as_float(v[c][2 * e2]), __uint_as_float(v[c][2 * e2 + 1])),
+                               SC, nl2[16 * c + e2]),
+                        x0, x1);
+              float p0, p1;
+              if ((e2 & 7) >= 5) {
+                exp2_poly5_x2(x0, x1, p0, p1);
+              } else {
+                p0 = fast_exp2(x0);
+                p1 = fast_exp2(x1);
               }
+              A[e2 & 3] = f2_add(A[e2 & 3], f2_pack(p0, p1));
             }
           }
-          if (!ok) { *s_abort = 1; break; }
-          float a0, a1, a2, a3;
-          f2_unpack(f2_add(A[0], A[1]), a0, a1);
-          f2_unpack(f2_add(A[2], A[3]), a2, a3);
-          const float acc = (a0 + a1) + (a2 + a3);
-          // add the two warpgroups' halves (exchange slot double-buffered by block
-          // parity, guarded by bounded mbarrier waits) and write the pooled value
-          const int sl = it & 1;
-          float* slot = red + sl * kTile;
-          if (w == 1) {
-            if (it >= 2 && !mbar_wait(bar(kPBarRedEmpty + sl), ((it >> 1) - 1) & 1, a.status)) { *s_abort = 1; break; }
-            slot[key] = acc;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(kPBarRedFull + sl));
-          } else {
-            if (!mbar_wait(bar(kPBarRedFull + sl), (it >> 1) & 1, a.status)) { *s_abort = 1; break; }
-            const float tot = acc + slot[key];
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(kPBarRedEmpty + sl));
-            const int col = kTile * jb + key;
-            if (rd == 0) prow[col] = tot * inv_count;
-            else prow[col] += tot * inv_count;
+        };
+        bool ok = true;
+        if (g < hg) {
+          if (!(ok = mbar_wait(bar(kPBarS + g), it & 1, a.status)) || *s_abort) {
+            *s_abort = 1;
+            break;
           }
+          tc_fence_after();
+          const uint32_t tS = tmem + 128 * g + lane_base;
+          uint32_t v[2][32];
+          tmem_ld32(tS, v[0]);
+          tmem_ld32(tS + 32, v[1]);
+          tmem_wait_ld();
+          reg_fence32(v[0]);
+          reg_fence32(v[1]);
+          sum_half(v, 0);
+          tmem_ld32(tS + 64, v[0]);
+          tmem_ld32(tS + 96, v[1]);
+          tmem_wait_ld();
+          reg_fence32(v[0]);
+          reg_fence32(v[1]);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(kPBarFree + g));  // the tile may be refilled
+          sum_half(v, 64);
+        }
+        float a0, a1, a2, a3;
+        f2_unpack(f2_add(A[0], A[1]), a0, a1);
+        f2_unpack(f2_add(A[2], A[3]), a2, a3);
+        const float acc = (a0 + a1) + (a2 + a3);
+        // heads 1-3 hand their sums to head 0's warpgroup (slot double-buffered by
+        // block parity, guarded by bounded mbarrier waits), which writes pooled
+        const int sl = it & 1;
+        float* slot = red + sl * 3 * kTile;
+        if (g > 0) {
+          if (it >= 2 && !mbar_wait(bar(kPBarRedEmpty + sl), ((it >> 1) - 1) & 1, a.status)) { *s_abort = 1; break; }
+          slot[(g - 1) * kTile + key] = acc;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(kPBarRedFull + sl));
+        } else {
+          if (!mbar_wait(bar(kPBarRedFull + sl), (it >> 1) & 1, a.status)) { *s_abort = 1; break; }
+          const float tot = acc + slot[key] + slot[kTile + key] + slot[2 * kTile + key];
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(kPBarRedEmpty + sl));
+          const int col = kTile * jb + key;
+          if (rd == 0) prow[col] = tot * inv_count;
+          else prow[col] += tot * inv_count;
         }
       }
       __syncthreads();
@@ -730,10 +767,10 @@ cudaError_t launch_prefill_anchor(const PrefillParams& p, cudaStream_t st) {
   a.B = p.B; a.Hq = p.Hq; a.Hkv = p.Hkv; a.G = p.G; a.N = p.N; a.n_tiles = n_tiles;
   a.scale_log2 = (float)((double)p.scale * 1.4426950408889634);
   a.lse = p.lse; a.pooled = p.pooled; a.status = p.status;
-  cudaFuncAttributes fa;  // same setmaxnreg split as the attention kernel
+  cudaFuncAttributes fa;  // the setmaxnreg split assumes kPoolLaunchRegs at launch
   e = cudaFuncGetAttributes(&fa, prefill_pool_kernel);
   if (e != cudaSuccess) return e;
-  if (fa.numRegs != kLaunchRegs) return cudaErrorNotSupported;
+  if (fa.numRegs != kPoolLaunchRegs) return cudaErrorNotSupported;
   e = cudaFuncSetAttribute(prefill_pool_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPoolSmem);
   if (e != cudaSuccess) return e;
   dim3 grid(n_tiles - 1, p.Hkv, p.B);
