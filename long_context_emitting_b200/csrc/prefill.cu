@@ -37,6 +37,9 @@
 //   TMEM lanes, queries on columns, one 128-column TMEM tile per head), so a
 //   thread owns one key and sums exp2(s - lse2) over the tile's queries in
 //   registers (3 of 8 exponentials on the FMA pipe, the rest on the SFU).
+//   The -lse term enters through one extra K16 step of the MMA (ones on the
+//   key side, -lse/scale split into three bf16 parts on the query side), so
+//   the summing loop reads no per-query values from shared memory.
 //   Warp roles (640 threads): a TMA producer and an MMA issuer in warpgroup 0,
 //   and four summing warpgroups, one per head of the round; a head's tile goes
 //   back to the MMA as soon as its scores are in registers.  The heads' sums
@@ -91,8 +94,13 @@ static_assert((kPoolLaunchRegs - kPoolCtlRegs) * 128 >= (kPoolSumRegs - kPoolLau
 static_assert(kPoolLaunchRegs * kPoolThreads <= 65536, "launch registers exceed the SM");
 constexpr uint32_t kPoolQ = 0;
 constexpr uint32_t kPoolK = kPoolHeads * kTileBytes;    // 2 stages
-constexpr uint32_t kPoolLse = kPoolK + 2 * kTileBytes;  // [kPoolHeads][128] floats
-constexpr uint32_t kPoolRed = kPoolLse + kPoolHeads * kTile * 4;  // [2 slots][3 heads][128] floats
+// One extra K16 step folds -lse into the MMA: K-side rows [1, 1, 1, 0 ...],
+// query-side rows [-v_hi, -v_mid, -v_lo, 0 ...] with v = lse / scale split into
+// three bf16 terms (32-byte-swizzled K-major tiles of 128 rows x 16).
+constexpr uint32_t kXBytes = 128u * 32u;
+constexpr uint32_t kPoolKx = kPoolK + 2 * kTileBytes;
+constexpr uint32_t kPoolQx = kPoolKx + kXBytes;         // [kPoolHeads] tiles
+constexpr uint32_t kPoolRed = kPoolQx + kPoolHeads * kXBytes;  // [2 slots][3 heads][128] floats
 constexpr uint32_t kPoolMisc = kPoolRed + 2 * 3 * kTile * 4;
 constexpr uint32_t kPoolSmem = kPoolMisc + 256 + 1024;
 // per head of the round: S^T tile full (MMA commit) / free (read into registers,
@@ -117,6 +125,7 @@ struct AttnArgs {
 struct PoolArgs {
   int B, Hq, Hkv, G, N, n_tiles;
   float scale_log2;
+  float inv_scale;  // 1 / scale
   const float* lse;
   float* pooled;
   unsigned* status;
@@ -486,7 +495,6 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  float* lse2 = reinterpret_cast<float*>(smem + kPoolLse);
   float* red = reinterpret_cast<float*>(smem + kPoolRed);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kPoolMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + kPoolMisc + 224);
@@ -520,13 +528,30 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   const uint32_t tmem = *tmem_slot;
   float* prow = a.pooled + (((int64_t)b * a.n_tiles + t) * a.Hkv + h) * a.N;
   const float inv_count = 1.f / (float)(kTile * G);
-  // -lse of a round's heads (log2 domain), read in pairs by the summing warps;
-  // every thread loads its share, then the CTA synchronises
-  auto load_lse2 = [&](int hg, int gbase) {
+  // The extra K16 step: the K side once per CTA, the query side of a round's
+  // heads from their log-sum-exp (every thread writes its share, then the CTA
+  // synchronises; the tensor cores read these through the async proxy).
+  for (int r = tid; r < kTile; r += kPoolThreads) {
+    const uint32_t one = 0x3F80u;  // bf16 1.0
+    *reinterpret_cast<uint4*>(smem + kPoolKx + sw32_chunk_offset(r, 0)) =
+        make_uint4(one | (one << 16), one, 0u, 0u);
+    *reinterpret_cast<uint4*>(smem + kPoolKx + sw32_chunk_offset(r, 1)) = make_uint4(0u, 0u, 0u, 0u);
+  }
+  auto load_lse = [&](int hg, int gbase) {
     for (int e = tid; e < hg * kTile; e += kPoolThreads) {
       const int j = e / kTile, q = e % kTile;
-      lse2[e] = -a.lse[((int64_t)b * a.Hq + gbase + j) * a.N + (int64_t)kTile * t + q] * kLog2e;
+      const float lse = a.lse[((int64_t)b * a.Hq + gbase + j) * a.N + (int64_t)kTile * t + q];
+      const float nv = -lse * a.inv_scale;  // the MMA adds -v to q.k; x = scale log2(e) (q.k - v)
+      const uint16_t hi = to_bf16_bits(nv);
+      const float r1 = nv - __uint_as_float((uint32_t)hi << 16);
+      const uint16_t mid = to_bf16_bits(r1);
+      const uint16_t lo = to_bf16_bits(r1 - __uint_as_float((uint32_t)mid << 16));
+      uint8_t* row = smem + kPoolQx + j * kXBytes;
+      *reinterpret_cast<uint4*>(row + sw32_chunk_offset(q, 0)) =
+          make_uint4((uint32_t)hi | ((uint32_t)mid << 16), (uint32_t)lo, 0u, 0u);
+      *reinterpret_cast<uint4*>(row + sw32_chunk_offset(q, 1)) = make_uint4(0u, 0u, 0u, 0u);
     }
+    fence_proxy_async_smem();
     __syncthreads();
   };
   // Each role runs its own copy of the round loop, so the compiler sizes every
@@ -537,7 +562,7 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       const int hg = min(kPoolHeads, G - rd * kPoolHeads);  // heads this round
       const int gbase = h * G + rd * kPoolHeads;
       const int it0 = rd * nblk;  // running block counter for stage / phase bookkeeping
-      load_lse2(hg, gbase);
+      load_lse(hg, gbase);
       if (warp == 0) {
         // ---------------------------- TMA producer ----------------------------
         if (lane == 0) {
@@ -575,6 +600,7 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
               for (int k16 = 0; k16 < 8; ++k16)
                 umma_ss(tmem + 128 * g, dk + kmajor_step(k16), dq + kmajor_step(k16), idesc, k16 > 0 ? 1u : 0u);
+              umma_ss(tmem + 128 * g, sw32_desc(sbase + kPoolKx), sw32_desc(sbase + kPoolQx + g * kXBytes), idesc, 1u);
               umma_commit(bar(kPBarS + g));
             }
             if (!ok) break;
@@ -584,7 +610,7 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           if (!ok) *s_abort = 1;
         }
       }
-      __syncthreads();  // round done: Q tiles and lse2 may be replaced
+      __syncthreads();  // round done: Q tiles and the -lse tiles may be replaced
     }
   } else {
     setmaxnreg_inc<kPoolSumRegs>();
@@ -600,21 +626,19 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       const int hg = min(kPoolHeads, G - rd * kPoolHeads);
       const int gbase = h * G + rd * kPoolHeads;
       const int it0 = rd * nblk;
-      load_lse2(hg, gbase);
+      load_lse(hg, gbase);
       for (int jb = 0; jb < nblk; ++jb) {
         const int it = it0 + jb;
         uint64_t A[4] = {0ull, 0ull, 0ull, 0ull};
-        // sum over 64 queries of exp2(s * sc - lse2), two per packed instruction;
-        // 3 of every 8 pairs on the FMA pipe, the rest on the SFU
-        auto sum_half = [&](const uint32_t (&v)[2][32], int q0) {
-          const uint64_t* nl2 = reinterpret_cast<const uint64_t*>(lse2 + g * kTile + q0);
+        // sum over 64 queries of exp2(sc * (q.k - lse/scale)), two per packed
+        // instruction; 3 of every 8 pairs on the FMA pipe, the rest on the SFU
+        auto sum_half = [&](const uint32_t (&v)[2][32]) {
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
 #pragma unroll
             for (int e2 = 0; e2 < 16; ++e2) {
               float x0, x1;
-              f2_unpack(f2_fma(f2_pack(__uint_as_float(v[c][2 * e2]), __uint_as_float(v[c][2 * e2 + 1])),
-                               SC, nl2[16 * c + e2]),
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(v[c][2 * e2]), __uint_as_float(v[c][2 * e2 + 1])), SC),
                         x0, x1);
               float p0, p1;
               if ((e2 & 7) >= 5) {
@@ -641,7 +665,7 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           tmem_wait_ld();
           reg_fence32(v[0]);
           reg_fence32(v[1]);
-          sum_half(v, 0);
+          sum_half(v);
           tmem_ld32(tS + 64, v[0]);
           tmem_ld32(tS + 96, v[1]);
           tmem_wait_ld();
@@ -650,7 +674,7 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(kPBarFree + g));  // the tile may be refilled
-          sum_half(v, 64);
+          sum_half(v);
         }
         float a0, a1, a2, a3;
         f2_unpack(f2_add(A[0], A[1]), a0, a1);
@@ -766,6 +790,7 @@ cudaError_t launch_prefill_anchor(const PrefillParams& p, cudaStream_t st) {
   PoolArgs a;
   a.B = p.B; a.Hq = p.Hq; a.Hkv = p.Hkv; a.G = p.G; a.N = p.N; a.n_tiles = n_tiles;
   a.scale_log2 = (float)((double)p.scale * 1.4426950408889634);
+  a.inv_scale = (float)(1.0 / (double)p.scale);
   a.lse = p.lse; a.pooled = p.pooled; a.status = p.status;
   cudaFuncAttributes fa;  // the setmaxnreg split assumes kPoolLaunchRegs at launch
   e = cudaFuncGetAttributes(&fa, prefill_pool_kernel);

@@ -291,6 +291,23 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo_byte
   return d;
 }
 
+// Descriptor for a K-major operand in the 32-byte-swizzled layout: rows of 32
+// bytes (one K16 step of bf16), 8-row groups of 256 bytes, the two 16-byte
+// chunks of row r swapped when bit 2 of r is set.  Base 256-byte aligned.
+__device__ __forceinline__ uint64_t sw32_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3fffu);
+  d |= (uint64_t)1 << 16;                  // leading offset: unused for swizzled K-major
+  d |= (uint64_t)(256u >> 4) << 32;        // 8-row group stride
+  d |= (uint64_t)1 << 46;                  // descriptor version for sm_100
+  d |= (uint64_t)6 << 61;                  // SWIZZLE_32B
+  return d;
+}
+// Byte offset of 16-byte chunk c (0 or 1) of row r in that layout.
+__host__ __device__ constexpr uint32_t sw32_chunk_offset(int r, int c) {
+  return (uint32_t)(r >> 3) * 256u + (uint32_t)(r & 7) * 32u + (uint32_t)((c ^ ((r >> 2) & 1)) * 16);
+}
+
 // Instruction descriptor: kind::f16, bf16 x bf16 -> fp32, M x N, operand majors.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
   return (1u << 4)                       // D format: f32
