@@ -92,6 +92,8 @@ constexpr int kPoolLaunchRegs = 96, kPoolSumRegs = 104, kPoolCtlRegs = 64;
 static_assert((kPoolLaunchRegs - kPoolCtlRegs) * 128 >= (kPoolSumRegs - kPoolLaunchRegs) * 512,
               "summing register increase must fit in what warpgroup 0 releases");
 static_assert(kPoolLaunchRegs * kPoolThreads <= 65536, "launch registers exceed the SM");
+// Q tiles as [64-dimension half][head][128 rows][128 B]: the rows of two
+// consecutive heads are contiguous, so a pair of heads is one N = 256 operand.
 constexpr uint32_t kPoolQ = 0;
 constexpr uint32_t kPoolK = kPoolHeads * kTileBytes;    // 2 stages
 // One extra K16 step folds -lse into the MMA: K-side rows [1, 1, 1, 0 ...],
@@ -105,6 +107,7 @@ constexpr uint32_t kPoolMisc = kPoolRed + 2 * 3 * kTile * 4;
 constexpr uint32_t kPoolSmem = kPoolMisc + 256 + 1024;
 // per head of the round: S^T tile full (MMA commit) / free (read into registers,
 // one arrival per warp); partial-sum exchange: heads 1-3 -> head 0's warpgroup
+// S / free per pair of heads (a single head when the group has one)
 enum { kPBarQ = 0, kPBarKFull = 1, kPBarKEmpty = 3, kPBarS = 5, kPBarFree = 9, kPBarRedFull = 13,
        kPBarRedEmpty = 15, kPoolBars = 17 };
 
@@ -145,6 +148,10 @@ __device__ __forceinline__ constexpr uint64_t kmajor_step(int ks) {
   return (uint64_t)(((uint32_t)(ks >> 2) * kHalfBytes + (uint32_t)(ks & 3) * 32u) >> 4);
 }
 __device__ __forceinline__ constexpr uint64_t mnmajor_step(int ks) { return (uint64_t)(ks * 2048u >> 4); }
+// k-step of the pooling kernel's [64-dim half][head][rows] Q layout
+__device__ __forceinline__ constexpr uint64_t qpair_step(int ks) {
+  return (uint64_t)(((uint32_t)(ks >> 2) * 4u * kHalfBytes + (uint32_t)(ks & 3) * 32u) >> 4);
+}
 
 template <bool GATHER>
 __global__ void __launch_bounds__(kAttnThreads, 1)
@@ -512,7 +519,11 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   if (tid == 0) {
     for (int i = 0; i < kPoolBars; ++i) {
       // free: the head's 4 warps; exchange full: 12 warps of heads 1-3; empty: head 0's 4 warps
-      const uint32_t count = (i >= kPBarRedFull && i < kPBarRedEmpty) ? 12u : (i >= kPBarFree ? 4u : 1u);
+      // free: the warps of the pair's (or single head's) warpgroups; exchange full:
+      // 12 warps of heads 1-3; exchange empty: head 0's 4 warps
+      const uint32_t n_free = G >= 2 ? 8u : 4u;
+      const uint32_t count = (i >= kPBarRedFull && i < kPBarRedEmpty) ? 12u
+                             : (i >= kPBarRedEmpty ? 4u : (i >= kPBarFree ? n_free : 1u));
       mbar_init(bar(i), count);
     }
     *s_abort = 0;
@@ -569,8 +580,8 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           mbar_expect_tx(bar(kPBarQ), hg * kTileBytes);
           for (int j = 0; j < hg; ++j) {
             const int y = (int)(((int64_t)b * a.Hq + gbase + j) * a.N + (int64_t)kTile * t);
-            tma_load_2d(sbase + kPoolQ + j * kTileBytes, &tm_q, 0, y, bar(kPBarQ));
-            tma_load_2d(sbase + kPoolQ + j * kTileBytes + kHalfBytes, &tm_q, 64, y, bar(kPBarQ));
+            tma_load_2d(sbase + kPoolQ + j * kHalfBytes, &tm_q, 0, y, bar(kPBarQ));
+            tma_load_2d(sbase + kPoolQ + (kPoolHeads + j) * kHalfBytes, &tm_q, 64, y, bar(kPBarQ));
           }
           for (int jb = 0; jb < nblk; ++jb) {
             const int it = it0 + jb, st = it & 1;
@@ -584,24 +595,27 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
       } else if (warp == 1) {
         // ---------------------------- MMA issuer ------------------------------
-        // S^T_g = K Q_g^T for each head g of the round into its own 128 TMEM
-        // columns, as soon as the summing warps have read that head's previous tile.
+        // S^T = K [Q_g; Q_g+1]^T for each pair of heads of the round (N = 256; a
+        // single head uses N = 128) into TMEM columns 128 g .., as soon as both
+        // heads' summing warps have read the pair's previous tile.
         if (lane == 0) {
-          const uint32_t idesc = idesc_bf16(128, 128, false, false);
+          const int np = hg >= 2 ? hg / 2 : 1;
+          const uint32_t idesc = idesc_bf16(128, hg >= 2 ? 256 : 128, false, false);
           bool ok = mbar_wait(bar(kPBarQ), rd & 1, a.status);
           for (int jb = 0; ok && jb < nblk; ++jb) {
             const int it = it0 + jb, st = it & 1;
             if (!(ok = mbar_wait(bar(kPBarKFull + st), (it >> 1) & 1, a.status))) break;
             const uint64_t dk = kmajor_desc(sbase + kPoolK + st * kTileBytes, 0);
-            for (int g = 0; g < hg; ++g) {
-              if (it >= 1 && !(ok = mbar_spin(bar(kPBarFree + g), (it - 1) & 1, a.status))) break;
+            for (int pr = 0; pr < np; ++pr) {
+              if (it >= 1 && !(ok = mbar_spin(bar(kPBarFree + pr), (it - 1) & 1, a.status))) break;
               tc_fence_after();
-              const uint64_t dq = kmajor_desc(sbase + kPoolQ + g * kTileBytes, 0);
+              const uint64_t dq = kmajor_desc(sbase + kPoolQ + 2 * pr * kHalfBytes, 0);
 #pragma unroll
               for (int k16 = 0; k16 < 8; ++k16)
-                umma_ss(tmem + 128 * g, dk + kmajor_step(k16), dq + kmajor_step(k16), idesc, k16 > 0 ? 1u : 0u);
-              umma_ss(tmem + 128 * g, sw32_desc(sbase + kPoolKx), sw32_desc(sbase + kPoolQx + g * kXBytes), idesc, 1u);
-              umma_commit(bar(kPBarS + g));
+                umma_ss(tmem + 256 * pr, dk + kmajor_step(k16), dq + qpair_step(k16), idesc, k16 > 0 ? 1u : 0u);
+              umma_ss(tmem + 256 * pr, sw32_desc(sbase + kPoolKx), sw32_desc(sbase + kPoolQx + 2 * pr * kXBytes),
+                      idesc, 1u);
+              umma_commit(bar(kPBarS + pr));
             }
             if (!ok) break;
             umma_commit(bar(kPBarKEmpty + st));
@@ -653,7 +667,7 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         };
         bool ok = true;
         if (g < hg) {
-          if (!(ok = mbar_wait(bar(kPBarS + g), it & 1, a.status)) || *s_abort) {
+          if (!(ok = mbar_wait(bar(kPBarS + g / 2), it & 1, a.status)) || *s_abort) {
             *s_abort = 1;
             break;
           }
@@ -673,7 +687,7 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           reg_fence32(v[1]);
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar(kPBarFree + g));  // the tile may be refilled
+          if (lane == 0) mbar_arrive(bar(kPBarFree + g / 2));  // the tile may be refilled
           sum_half(v);
         }
         float a0, a1, a2, a3;
