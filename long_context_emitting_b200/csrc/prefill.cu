@@ -641,6 +641,23 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       const int gbase = h * G + rd * kPoolHeads;
       const int it0 = rd * nblk;
       load_lse(hg, gbase);
+      float pend = 0.f;  // head 0's warpgroup: its own sum of the previous block
+      // adds heads 1-3 of block itp (block jbp of the round) to `mine`, writes pooled
+      auto combine = [&](int rdp, int itp, int jbp, float mine) -> bool {
+        const int sl = itp & 1;
+        if (!mbar_wait(bar(kPBarRedFull + sl), (itp >> 1) & 1, a.status)) {
+          *s_abort = 1;
+          return false;
+        }
+        const float* slot = red + sl * 3 * kTile;
+        const float tot = mine + slot[key] + slot[kTile + key] + slot[2 * kTile + key];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kPBarRedEmpty + sl));
+        const int col = kTile * jbp + key;
+        if (rdp == 0) prow[col] = tot * inv_count;
+        else prow[col] += tot * inv_count;
+        return true;
+      };
       for (int jb = 0; jb < nblk; ++jb) {
         const int it = it0 + jb;
         uint64_t A[4] = {0ull, 0ull, 0ull, 0ull};
@@ -694,25 +711,23 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         f2_unpack(f2_add(A[0], A[1]), a0, a1);
         f2_unpack(f2_add(A[2], A[3]), a2, a3);
         const float acc = (a0 + a1) + (a2 + a3);
-        // heads 1-3 hand their sums to head 0's warpgroup (slot double-buffered by
-        // block parity, guarded by bounded mbarrier waits), which writes pooled
-        const int sl = it & 1;
-        float* slot = red + sl * 3 * kTile;
+        // Heads 1-3 hand their sums to head 0's warpgroup through shared memory
+        // (slot double-buffered by block parity, guarded by bounded mbarrier
+        // waits).  Head 0's warpgroup adds them one block late, while its own
+        // next block is under way, so it never waits for the slowest head.
         if (g > 0) {
+          const int sl = it & 1;
           if (it >= 2 && !mbar_wait(bar(kPBarRedEmpty + sl), ((it >> 1) - 1) & 1, a.status)) { *s_abort = 1; break; }
-          slot[(g - 1) * kTile + key] = acc;
+          red[(sl * 3 + g - 1) * kTile + key] = acc;
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(kPBarRedFull + sl));
         } else {
-          if (!mbar_wait(bar(kPBarRedFull + sl), (it >> 1) & 1, a.status)) { *s_abort = 1; break; }
-          const float tot = acc + slot[key] + slot[kTile + key] + slot[2 * kTile + key];
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(kPBarRedEmpty + sl));
-          const int col = kTile * jb + key;
-          if (rd == 0) prow[col] = tot * inv_count;
-          else prow[col] += tot * inv_count;
+          if (jb > 0 && !(ok = combine(rd, it - 1, jb - 1, pend))) break;
+          pend = acc;
         }
       }
+      // head 0's warpgroup: the round's last block
+      if (g == 0 && nblk > 0 && !*s_abort) combine(rd, it0 + nblk - 1, nblk - 1, pend);
       __syncthreads();
     }
   }
