@@ -14,7 +14,8 @@
 //                 anchor: dense key blocks 0..t (block t is the diagonal);
 //                 reuse: the anchor's indices of row (t, head_map[h]) gathered
 //                 with cp.async (two whole rows per warp instruction) into the
-//                 same swizzled layout, then the diagonal block by TMA.
+//                 same swizzled layout by warps 8, 10 and 11 together, then the
+//                 diagonal block by TMA.
 //     warp 9      MMA issuer (one thread): S_i = Q_i K^T into TMEM, and
 //                 O_i += P_i V with P_i read from TMEM (it overwrites S_i).
 //     warps 0-7   softmax, one warpgroup per tile, one query row (TMEM lane)
@@ -67,8 +68,9 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ---- attention kernel layout ----
-constexpr int kAttnThreads = 384;  // softmax warps 0-7, producer warp 8, MMA warp 9 (10, 11 idle)
+constexpr int kAttnThreads = 384;  // softmax warps 0-7, producer warp 8, MMA warp 9, 10-11 gather helpers
 constexpr int kProducerWarp = 8, kMmaWarp = 9;
+constexpr int kGatherWarps = 3;    // reuse: warps 8, 10 and 11 share the row gathers of a block
 // setmaxnreg split: the launch gives every thread kLaunchRegs (the compiler's
 // count, checked on the host); the third warpgroup releases down to kOtherRegs
 // and the two softmax warpgroups take exactly what it releases.
@@ -199,7 +201,8 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   if (tid == 0) {
     for (int i = 0; i < kAttnBars; ++i) {
       const bool per_warp = i >= kBarP && i < kBarP + 4;  // 4 softmax warps per tile
-      mbar_init(bar(i), per_warp ? 4u : 1u);
+      const bool kv_full = i >= kBarKvFull && i < kBarKvFull + 2;  // reuse: one arrival per gather warp
+      mbar_init(bar(i), per_warp ? 4u : (kv_full && GATHER ? (uint32_t)kGatherWarps : 1u));
     }
     *s_abort = 0;
     mbar_fence_init();
@@ -215,9 +218,11 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
   if (warp >= 8) {
     setmaxnreg_dec<kOtherRegs>();
-  if (warp == kProducerWarp) {
+    // gather warp index: producer warp 8 is 0, warps 10 and 11 are 1 and 2 (reuse only)
+    const int gw = warp == kProducerWarp ? 0 : (warp >= 10 ? warp - 9 : -1);
+    if (gw == 0 || (GATHER && gw > 0)) {
       // ================================ TMA producer ================================
-      if (lane == 0) {
+      if (gw == 0 && lane == 0) {
         mbar_expect_tx(bar(kBarQ), ntile * kTileBytes);
         for (int i = 0; i < ntile; ++i) {
           const int y = (int)(q_row0 + (int64_t)i * a.N);
@@ -233,7 +238,9 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const uint32_t vb = kb + kTileBytes;
         const bool dense = !GATHER || j == n_gather;
         if (dense) {
-          if (lane == 0) {
+          if (gw > 0) {
+            if (lane == 0) mbar_arrive(bar(kBarKvFull + st));  // helpers complete the count
+          } else if (lane == 0) {
             mbar_expect_tx(bar(kBarKvFull + st), 2 * kTileBytes);
             const int y = kv_row0 + kTile * (GATHER ? t : j);
             tma_load_2d(kb, &tm_k, 0, y, bar(kBarKvFull + st));
@@ -243,21 +250,24 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           }
         } else {
           // Gathered block: validity of rows 32e + lane -> ballot word e (bit = row & 31).
-          uint32_t m[4];
+          uint32_t m[4] = {0u, 0u, 0u, 0u};
+          if (gw == 0) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int pos = kTile * j + 32 * e + lane;
-            const int key = pos < kt ? __ldg(irow + pos) : -1;
-            const bool ok = key >= 0 && key < kTile * t;
-            if (pos < kt && !ok) flag_status(a.status, kStatusBadIndex);
-            m[e] = __ballot_sync(0xffffffffu, ok);
+            for (int e = 0; e < 4; ++e) {
+              const int pos = kTile * j + 32 * e + lane;
+              const int key = pos < kt ? __ldg(irow + pos) : -1;
+              const bool ok = key >= 0 && key < kTile * t;
+              if (pos < kt && !ok) flag_status(a.status, kStatusBadIndex);
+              m[e] = __ballot_sync(0xffffffffu, ok);
+            }
           }
           // Copy: each warp instruction moves two whole 256-byte rows (16 lanes per
           // row, one 16-byte chunk each) into the swizzled layout; masked rows are
-          // zero-filled from a valid address.
+          // zero-filled from a valid address.  The gather warps take every third
+          // pair of rows.
           const int c16 = lane & 15;
           const uint32_t half = (uint32_t)(c16 >> 3) * kHalfBytes;
-          for (int s2 = 0; s2 < kTile / 2; ++s2) {
+          for (int s2 = gw; s2 < kTile / 2; s2 += kGatherWarps) {
             const int row = 2 * s2 + (lane >> 4);
             const int pos = kTile * j + row;
             const int key = pos < kt ? __ldg(irow + pos) : -1;
@@ -272,9 +282,11 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           fence_proxy_async_smem();  // the tensor cores read these rows through the async proxy
           __syncwarp();
           if (lane == 0) {
+            if (gw == 0) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) masks[st * 4 + e] = m[e];
-            mbar_arrive(bar(kBarKvFull + st));  // release: rows and masks visible
+              for (int e = 0; e < 4; ++e) masks[st * 4 + e] = m[e];
+            }
+            mbar_arrive(bar(kBarKvFull + st));  // release: rows (and masks) visible
           }
         }
       }
