@@ -54,9 +54,9 @@ def parse():
 # call's kernels) from the ncu capture summarised in the named profile; set an
 # entry to None when one of its kernels changes until it is captured again.
 NCU_TRAFFIC = {
-    "prefill_anchor": {"bytes": 299933440 + 187733248,
+    "prefill_anchor": {"bytes": 300512512 + 187554304,
                        "profile": "profiles/traffic_prefill_n16384_decode_b16_t32768.md"},
-    "decode_anchor": {"bytes": 2147662848 + 24422400 + 75660800 + 197376,
+    "decode_anchor": {"bytes": 2147660032 + 24662784 + 75661056 + 187648,
                       "profile": "profiles/traffic_prefill_n16384_decode_b16_t32768.md"},
 }
 

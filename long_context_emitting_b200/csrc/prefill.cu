@@ -65,7 +65,6 @@ constexpr uint32_t kHalfBytes = 128u * 128u;     // 64 bf16 columns x 128 rows (
 constexpr uint32_t kTileBytes = 2u * kHalfBytes;  // 128 x 128 bf16
 constexpr float kRescaleLog2 = 8.f;
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kLog2e = 1.4426950408889634f;
 
 // ---- attention kernel layout ----
 constexpr int kAttnThreads = 384;  // softmax warps 0-7, producer warp 8, MMA warp 9, 10-11 gather helpers
@@ -694,9 +693,8 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
           }
         };
-        bool ok = true;
         if (g < hg) {
-          if (!(ok = mbar_wait(bar(kPBarS + g / 2), it & 1, a.status)) || *s_abort) {
+          if (!mbar_wait(bar(kPBarS + g / 2), it & 1, a.status) || *s_abort) {
             *s_abort = 1;
             break;
           }
@@ -734,7 +732,7 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(kPBarRedFull + sl));
         } else {
-          if (jb > 0 && !(ok = combine(rd, it - 1, jb - 1, pend))) break;
+          if (jb > 0 && !combine(rd, it - 1, jb - 1, pend)) break;
           pend = acc;
         }
       }
