@@ -53,6 +53,8 @@ def parse():
 # DRAM bytes per call (dram__bytes_read.sum + dram__bytes_write.sum of the
 # call's kernels) from the ncu capture summarised in the named profile; set an
 # entry to None when one of its kernels changes until it is captured again.
+# (The pooling kernel's exp split between SFU and FMA pipe changed after the
+# capture; that moves no memory traffic.)
 NCU_TRAFFIC = {
     "prefill_anchor": {"bytes": 300512512 + 187554304,
                        "profile": "profiles/traffic_prefill_n16384_decode_b16_t32768.md"},

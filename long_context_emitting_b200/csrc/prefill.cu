@@ -37,7 +37,7 @@
 //   the tile it computes S^T = K Q_g^T for the group's query heads (keys on
 //   TMEM lanes, queries on columns, one 128-column TMEM tile per head), so a
 //   thread owns one key and sums exp2(s - lse2) over the tile's queries in
-//   registers (3 of 8 exponentials on the FMA pipe, the rest on the SFU).
+//   registers (2 of 8 exponentials on the FMA pipe, the rest on the SFU).
 //   The -lse term enters through one extra K16 step of the MMA (ones on the
 //   key side, -lse/scale split into three bf16 parts on the query side), so
 //   the summing loop reads no per-query values from shared memory.
@@ -673,7 +673,7 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const int it = it0 + jb;
         uint64_t A[4] = {0ull, 0ull, 0ull, 0ull};
         // sum over 64 queries of exp2(sc * (q.k - lse/scale)), two per packed
-        // instruction; 3 of every 8 pairs on the FMA pipe, the rest on the SFU
+        // instruction; 2 of every 8 pairs on the FMA pipe, the rest on the SFU
         auto sum_half = [&](const uint32_t (&v)[2][32]) {
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
@@ -683,7 +683,7 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
               f2_unpack(f2_mul(f2_pack(__uint_as_float(v[c][2 * e2]), __uint_as_float(v[c][2 * e2 + 1])), SC),
                         x0, x1);
               float p0, p1;
-              if ((e2 & 7) >= 5) {
+              if ((e2 & 7) >= 6) {
                 exp2_poly5_x2(x0, x1, p0, p1);
               } else {
                 p0 = fast_exp2(x0);
