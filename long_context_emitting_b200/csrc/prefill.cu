@@ -229,8 +229,33 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           tma_load_2d(sbase + kAttnQ + i * kTileBytes + kHalfBytes, &tm_q, 64, y, bar(kBarQ));
         }
       }
+      // Reuse: the gathered rows of a layer are first read from DRAM at scattered
+      // positions; their latency would exceed a block's compute.  Each gather warp
+      // pulls its share of the rows of block j + 2 into L2 before it waits for
+      // the stage of block j, so the later copies are L2 hits.
+      auto prefetch_rows = [&](int jp) {
+        if constexpr (GATHER) {
+          if (jp >= n_gather) return;
+          for (int r = gw + kGatherWarps * lane; r < kTile; r += kGatherWarps * 32) {
+            const int pos = kTile * jp + r;
+            if (pos >= kt) break;
+            const int key = __ldg(irow + pos);
+            if (key < 0 || key >= kTile * t) continue;  // flagged when the block is gathered
+            const int64_t off = ((int64_t)kv_row0 + key) * kHeadDim;
+            prefetch_l2(a.k + off);
+            prefetch_l2(a.k + off + 64);
+            prefetch_l2(a.v + off);
+            prefetch_l2(a.v + off + 64);
+          }
+        }
+      };
+      if (GATHER) {
+        prefetch_rows(0);
+        prefetch_rows(1);
+      }
       for (int j = 0; j < nblk; ++j) {
         const int st = j & 1;
+        prefetch_rows(j + 2);
         if (j >= 2 && !mbar_wait(bar(kBarKvEmpty + st), ((j >> 1) - 1) & 1, a.status)) { *s_abort = 1; break; }
         if (*s_abort) break;
         const uint32_t kb = sbase + kAttnKV + (2 * st) * kTileBytes;
