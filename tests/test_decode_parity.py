@@ -87,6 +87,14 @@ def test_decode_small_ragged():
     _check_layer_pair(cfg)
 
 
+@pytest.mark.parametrize("Hq,Hkv", [(8, 8), (16, 8), (64, 8)])
+def test_decode_gqa_group_sizes(Hq, Hkv):
+    # G = 1, 2 and 8 query heads per KV head (padding rows of the mma tile for G < 8)
+    cfg = workload.scaled(workload.DECODE_4K, name=f"decode_g{Hq // Hkv}", B=3, T=None,
+                          T_list=(1, 300, 1029), Hq=Hq, Hkv=Hkv)
+    _check_layer_pair(cfg)
+
+
 def test_decode_b1_t4096_all_layers():
     cfg = workload.DECODE_4K
     lens = cfg.seq_lens()

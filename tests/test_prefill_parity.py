@@ -80,6 +80,14 @@ def test_prefill_small_all_tiles():
     _check(cfg)
 
 
+@pytest.mark.parametrize("Hq,Hkv", [(8, 8), (16, 8), (32, 4)])
+def test_prefill_gqa_group_sizes(Hq, Hkv):
+    # G = 1 (one tile per CTA; pooling with a single N = 128 head), G = 2 (one
+    # pair of heads), G = 8 (two pooling rounds of four heads)
+    cfg = workload.scaled(workload.PREFILL_16K, name=f"prefill_g{Hq // Hkv}", N=512, Hq=Hq, Hkv=Hkv)
+    _check(cfg)
+
+
 def test_prefill_batch2():
     cfg = workload.scaled(workload.PREFILL_16K, name="prefill_b2", N=384, B=2)
     _check(cfg, b=1)
