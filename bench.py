@@ -293,6 +293,56 @@ def prefill_step(sch, layers, maps, outs, timer=None):
 
 
 # --------------------------------------------------------------------------------------
+def calibration_timing(dev, reps: int = 20):
+    """Calibration parts (offline, outside the timed step) on decode-shaped
+    synthetic rows: 128 rows (16 sequences x 8 KV heads) of 32768 positions,
+    k = 3277.  Times one similarity launch (one layer pair), a whole head remap
+    (two Top-k launches, one similarity launch over the 64 head pairs) and the
+    anchor DP for 32 layers and 5 anchors (host code)."""
+    import time
+    import numpy as np
+    from long_context_emitting_b200 import api
+
+    g = torch.Generator(device=dev).manual_seed(20251218)
+    rows, n, k, Hkv = 128, 32768, 3277, 8
+    pa = torch.rand(rows, n, generator=g, device=dev) ** 8
+    pb = torch.rand(rows, n, generator=g, device=dev) ** 8
+    pa /= pa.sum(-1, keepdim=True)
+    pb /= pb.sum(-1, keepdim=True)
+    row_len = torch.full((rows,), n, dtype=torch.int32, device=dev)
+    row_k = torch.full((rows,), k, dtype=torch.int32, device=dev)
+    ia = api.topk(pa, row_len, row_k, k)
+    ib = api.topk(pb, row_len, row_k, k)
+    out = torch.empty(rows, dtype=torch.float64, device=dev)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(reps):
+            fn()
+        e.record()
+        torch.cuda.synchronize()
+        return s.elapsed_time(e) / reps * 1e3
+
+    sim_us = timed(lambda: api.similarity_rows(pb, row_len, row_k, ia, ib, out=out))
+    remap_us = timed(lambda: api.head_remap(pa.view(Hkv, rows // Hkv, n), pb.view(Hkv, rows // Hkv, n), k))
+    rng = np.random.default_rng(0)
+    S = np.triu(rng.random((32, 32)))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        api.select_anchors(S, 5)
+    dp_us = (time.perf_counter() - t0) / reps * 1e6
+    # algorithmic bytes of one similarity launch: two index lists and the two
+    # gathered values per selected position (4 B each)
+    sim_bytes = rows * k * 4 * 4
+    return {"workload": "128 rows x 32768, k=3277 (decode_b16_t32768 pooled shape), synthetic",
+            "similarity_rows_us": sim_us, "similarity_gbs": sim_bytes / (sim_us * 1e-6) / 1e9,
+            "head_remap_us": remap_us, "select_anchors_L32_M5_host_us": dp_us}
+
+
 def cpu_sample(steps: int = 1):
     """The float64 oracle on a bounded sample of the same workload (host cores).
 
@@ -597,6 +647,8 @@ def main():
     out["roofline"] = roofline
     out["clocks"] = clk
 
+    if dec and dist.rank == 0:
+        out["calibration"] = calibration_timing(dev)
     if not args.no_e2e:
         out["e2e"] = e2e(dec, pre, args, dist)
     if not args.no_cpu and dist.rank == 0:

@@ -196,6 +196,45 @@ int kascade_prefill_reuse(kascade_shape s, int32_t N, const uint16_t* q, const u
                           float* lse, void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------- */
+/* Calibration (Kascade explainer, レイヤー間類似度とアンカーレイヤー選択 and
+ * 動的計画法): which layers are anchors and which anchor KV head each reuse
+ * head follows are chosen offline from post-softmax distributions.
+ *
+ * kascade_similarity_rows: the sim ratio of the explainer per row, the share of
+ * layer b's Top-k probability mass that layer a's Top-k indices recover.  For
+ * output row r, with rb = b_row[r] (r if b_row is NULL) and ra = a_row[r]
+ * (r if a_row is NULL) and k = row_k[rb]:
+ *     ratio[r] = sum_{i<k} p_b[rb][idx_a[ra][i]] / sum_{i<k} p_b[rb][idx_b[rb][i]]
+ * (fp64 sums; 0 when the denominator is 0).  The row maps let one call compare
+ * every (anchor head, reuse head) pair without copying rows.
+ *   p_b       device fp32 [rows, ld], 16-byte aligned, ld % 4 == 0: layer b's rows
+ *   row_len   device int32 [rows]: valid length of each row (<= ld)
+ *   row_k     device int32 [rows]: k of each row (<= row_len, <= k_max)
+ *   idx_a     device int32 [rows, k_max]: layer a's Top-k indices (kascade_topk output)
+ *   idx_b     device int32 [rows, k_max]: layer b's Top-k indices
+ *   b_row, a_row  device int32 [n_out] or NULL: source rows of each output row
+ *   ratio     device fp64 [n_out]: output
+ * Indices or rows out of range are skipped and set KASCADE_ERR_BAD_INDEX in the
+ * device status.  Asynchronous on `stream`. */
+int kascade_similarity_rows(const float* p_b, int32_t rows, int64_t ld, const int32_t* row_len,
+                            const int32_t* row_k, const int32_t* idx_a, const int32_t* idx_b,
+                            int32_t k_max, int32_t n_out, const int32_t* b_row,
+                            const int32_t* a_row, double* ratio, void* stream);
+
+/* kascade_select_anchors: Algorithm 1 of the explainer on the HOST (no GPU
+ * work).  S is host fp64 [L, L] row-major, the weighted similarity matrix
+ * (S[i][l] = w_l * sim(i, l) for l >= i).  Chooses M anchor layers maximising
+ * sum_l S[a(l)][l], a(l) the last anchor at or before l, by
+ *     dp[m][j] = max_{i=m-1..j-1} dp[m-1][i] + sum_{l=i}^{j-1} S[i][l]
+ * with dp[0][0] = 0, dp[0][j>0] = -inf (so layer 0 is always an anchor), the
+ * smallest i kept among equal maxima; O(M L^2) time, O(M L + L^2) memory.
+ *   anchors   host int32 [M]: output, ascending
+ *   best      host fp64: output, dp[M][L]
+ * Returns KASCADE_ERR_INVALID_ARG unless 1 <= M <= L <= 4096 and the pointers
+ * are non-NULL; KASCADE_ERR_NONFINITE if S holds a NaN or an infinity. */
+int kascade_select_anchors(const double* S, int32_t L, int32_t M, int32_t* anchors, double* best);
+
+/* ------------------------------------------------------------------------- */
 /* Waits for `stream`, then returns and clears the sticky device status of the
  * current device: KASCADE_OK, or the first of KASCADE_ERR_BAD_INDEX /
  * KASCADE_ERR_NONFINITE that a kernel recorded (KASCADE_ERR_CUDA if the wait fails). */

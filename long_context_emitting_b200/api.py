@@ -183,5 +183,115 @@ def prefill_reuse(q, k, v, idx, idx_k, head_map, scale: float, out=None, lse=Non
     return out, lse
 
 
+# ----------------------------------------------------------- calibration ----
+def similarity_rows(p_b, row_len, row_k, idx_a, idx_b, b_row=None, a_row=None, out=None):
+    """Per-row similarity ratio (kascade_similarity_rows): fp64 [n_out].
+
+    Row r compares the Top-k set idx_a[a_row[r]] with idx_b[b_row[r]] on the
+    distribution p_b[b_row[r]] (identity maps when b_row / a_row are None).
+    """
+    _need_cuda("p_b", p_b, torch.float32)
+    for name, t in (("row_len", row_len), ("row_k", row_k), ("idx_a", idx_a), ("idx_b", idx_b)):
+        _need_cuda(name, t, torch.int32)
+    for name, t in (("b_row", b_row), ("a_row", a_row)):
+        if t is not None:
+            _need_cuda(name, t, torch.int32)
+    ld = p_b.shape[-1]
+    rows = p_b.numel() // ld if ld else 0
+    k_max = idx_a.shape[-1]
+    n_out = b_row.numel() if b_row is not None else rows
+    out = torch.empty(n_out, dtype=torch.float64, device=p_b.device) if out is None else out
+    rc = _lib().kascade_similarity_rows(_ptr(p_b), int(rows), int(ld), _ptr(row_len), _ptr(row_k),
+                                        _ptr(idx_a), _ptr(idx_b), int(k_max), int(n_out),
+                                        _ptr(b_row), _ptr(a_row), _ptr(out), _stream())
+    check(rc, "kascade_similarity_rows")
+    return out
+
+
+def _pad4(p):
+    """Rows padded to a multiple of 4 floats (the 16-byte row stride the kernels
+    require); the padding lies beyond every row's length and is never read."""
+    n = p.shape[-1]
+    if n % 4 == 0 and p.is_contiguous():
+        return p
+    out = torch.zeros(*p.shape[:-1], (n + 3) // 4 * 4, dtype=p.dtype, device=p.device)
+    out[..., :n] = p
+    return out
+
+
+def _row_sets(p, k, n):
+    """Top-k sets of every row of p [rows, >= n] over its first n entries."""
+    rows = p.shape[0]
+    row_len = torch.full((rows,), n, dtype=torch.int32, device=p.device)
+    row_k = torch.full((rows,), k, dtype=torch.int32, device=p.device)
+    return topk(p, row_len, row_k, k), row_len, row_k
+
+
+def similarity(p_a, p_b, k: int) -> float:
+    """sim(a, b) of two layers: the mean over rows (queries, or pooled rows) of
+    the share of b's Top-k mass that a's Top-k indices recover."""
+    n = p_a.shape[-1]
+    p_a, p_b = _pad4(p_a), _pad4(p_b)
+    ia, row_len, row_k = _row_sets(p_a, k, n)
+    ib, _, _ = _row_sets(p_b, k, n)
+    return float(similarity_rows(p_b, row_len, row_k, ia, ib).mean().item())
+
+
+def similarity_matrix(p_layers, k: int):
+    """L x L host fp64 matrix of sim(a, b) for a <= b (0 below the diagonal), from
+    per-layer distributions p_layers [L, rows, n] (one Top-k pass per layer)."""
+    L, n = p_layers.shape[0], p_layers.shape[-1]
+    p_layers = _pad4(p_layers)
+    sets = [_row_sets(p_layers[l], k, n) for l in range(L)]
+    sim = torch.zeros(L, L, dtype=torch.float64)
+    for a in range(L):
+        for b in range(a, L):
+            ib, row_len, row_k = sets[b]
+            r = similarity_rows(p_layers[b], row_len, row_k, sets[a][0], ib)
+            sim[a, b] = r.mean().item()
+    return sim.numpy()
+
+
+def head_remap(p_anchor, p_reuse, k: int):
+    """Reuse-layer KV head -> anchor KV head with the highest similarity.
+
+    p_anchor / p_reuse: [Hkv, Q, n] distributions.  One similarity launch covers
+    every (reuse head, anchor head) pair; ties go to the lower anchor head.
+    Returns int64 [Hkv] on the device.
+    """
+    Hkv, Q, n = p_anchor.shape
+    p_anchor, p_reuse = _pad4(p_anchor), _pad4(p_reuse)
+    ld = p_anchor.shape[-1]
+    ia, row_len, row_k = _row_sets(p_anchor.reshape(Hkv * Q, ld), k, n)
+    ib, _, _ = _row_sets(p_reuse.reshape(Hkv * Q, ld), k, n)
+    dev = p_anchor.device
+    h = torch.arange(Hkv, device=dev).view(Hkv, 1, 1)
+    a = torch.arange(Hkv, device=dev).view(1, Hkv, 1)
+    q = torch.arange(Q, device=dev).view(1, 1, Q)
+    b_row = (h * Q + q).expand(Hkv, Hkv, Q).reshape(-1).to(torch.int32).contiguous()
+    a_row = (a * Q + q).expand(Hkv, Hkv, Q).reshape(-1).to(torch.int32).contiguous()
+    r = similarity_rows(p_reuse.reshape(Hkv * Q, ld), row_len, row_k, ia, ib, b_row, a_row)
+    return r.view(Hkv, Hkv, Q).mean(-1).argmax(dim=1)
+
+
+def select_anchors(S, M: int):
+    """Anchor layers by the dynamic program (kascade_select_anchors, host code).
+
+    S: the L x L weighted similarity matrix (array-like, fp64).  Returns
+    (best covered similarity, ascending list of M anchor layers).
+    """
+    import ctypes
+    import numpy as np
+
+    S = np.ascontiguousarray(S, dtype=np.float64)
+    L = S.shape[0]
+    anchors = np.zeros(max(M, 1), dtype=np.int32)
+    best = ctypes.c_double(0.0)
+    rc = _lib().kascade_select_anchors(S.ctypes.data, int(L), int(M), anchors.ctypes.data,
+                                       ctypes.addressof(best))
+    check(rc, "kascade_select_anchors")
+    return best.value, [int(x) for x in anchors[:M]]
+
+
 def default_scale(d: int = HEAD_DIM) -> float:
     return 1.0 / math.sqrt(d)

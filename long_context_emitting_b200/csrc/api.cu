@@ -168,6 +168,36 @@ int kascade_topk(const float* scores, int32_t rows, int64_t ld, const int32_t* r
                                static_cast<cudaStream_t>(stream)));
 }
 
+// ------------------------------------------------------------- calibration --
+int kascade_similarity_rows(const float* p_b, int32_t rows, int64_t ld, const int32_t* row_len,
+                            const int32_t* row_k, const int32_t* idx_a, const int32_t* idx_b,
+                            int32_t k_max, int32_t n_out, const int32_t* b_row,
+                            const int32_t* a_row, double* ratio, void* stream) {
+  if (rows < 0 || ld < 0 || k_max < 0 || n_out < 0) return KASCADE_ERR_INVALID_ARG;
+  if (n_out == 0) return KASCADE_OK;
+  if (rows == 0 || !p_b || !row_len || !row_k || !ratio || (k_max > 0 && (!idx_a || !idx_b)))
+    return KASCADE_ERR_INVALID_ARG;
+  if (!aligned16(p_b) || (ld & 3) || ((uintptr_t)row_len & 3) || ((uintptr_t)row_k & 3) ||
+      ((uintptr_t)idx_a & 3) || ((uintptr_t)idx_b & 3) || ((uintptr_t)b_row & 3) ||
+      ((uintptr_t)a_row & 3) || ((uintptr_t)ratio & 7))
+    return KASCADE_ERR_INVALID_ARG;
+  unsigned* st = device_status_ptr();
+  if (!st) return KASCADE_ERR_CUDA;
+  SimArgs a;
+  a.p_b = p_b; a.rows = rows; a.ld = ld; a.row_len = row_len; a.row_k = row_k;
+  a.idx_a = idx_a; a.idx_b = idx_b; a.k_max = k_max; a.b_row = b_row; a.a_row = a_row;
+  a.ratio = ratio; a.status = st;
+  return from_cuda(launch_similarity_rows(a, n_out, static_cast<cudaStream_t>(stream)));
+}
+
+int kascade_select_anchors(const double* S, int32_t L, int32_t M, int32_t* anchors, double* best) {
+  if (!S || !anchors || !best || L < 1 || L > 4096 || M < 1 || M > L) return KASCADE_ERR_INVALID_ARG;
+  for (int64_t i = 0; i < (int64_t)L * L; ++i)
+    if (!std::isfinite(S[i])) return KASCADE_ERR_NONFINITE;
+  select_anchors_dp(S, L, M, anchors, best);
+  return KASCADE_OK;
+}
+
 // ----------------------------------------------------------------- prefill --
 static int check_prefill(const kascade_shape& s, int32_t N) {
   int rc = check_shape(s);

@@ -1,0 +1,125 @@
+// Calibration parts of Kascade: the cross-layer similarity ratio on the GPU
+// and the anchor-selection dynamic program on the host.
+//
+// Method: Kascade explainer (0h-n0.github.io), レイヤー間類似度とアンカーレイヤー選択
+// (the sim equation: the share of layer b's Top-k probability mass that layer
+// a's Top-k indices recover) and 動的計画法 (Algorithm 1: choose M anchor layers
+// maximising the covered weighted similarity, O(M L^2)).
+//
+// similarity_rows_kernel
+//   One CTA per output row r.  With rb = b_row[r] (or r) and ra = a_row[r] (or
+//   r) it sums, in fp64, P_b[rb, idx_a[ra, i]] and P_b[rb, idx_b[rb, i]] over
+//   i < k = row_k[rb], and writes their ratio.  The index lists are the Top-k
+//   outputs of layers a and b; indices outside [0, row_len[rb]) are skipped and
+//   flagged in the device status.
+#include "common.cuh"
+#include "internal.h"
+
+#include <cmath>
+#include <vector>
+
+namespace kascade {
+
+namespace {
+
+constexpr int kSimThreads = 256;
+
+__global__ void __launch_bounds__(kSimThreads) similarity_rows_kernel(const SimArgs a) {
+  __shared__ double s_num[kSimThreads / 32], s_den[kSimThreads / 32];
+  const int r = blockIdx.x;
+  const int rb = a.b_row ? a.b_row[r] : r;
+  const int ra = a.a_row ? a.a_row[r] : r;
+  double num = 0.0, den = 0.0;
+  bool bad = rb < 0 || rb >= a.rows || ra < 0 || ra >= a.rows;
+  if (!bad) {
+    const int len = a.row_len[rb];
+    const int k = a.row_k[rb];
+    if (len < 0 || (int64_t)len > a.ld || k < 0 || k > len || k > a.k_max) {
+      bad = true;
+    } else {
+      const float* p = a.p_b + (int64_t)rb * a.ld;
+      const int32_t* ia = a.idx_a + (int64_t)ra * a.k_max;
+      const int32_t* ib = a.idx_b + (int64_t)rb * a.k_max;
+      for (int i = threadIdx.x; i < k; i += kSimThreads) {
+        const int ja = __ldg(ia + i), jb = __ldg(ib + i);
+        if (ja >= 0 && ja < len) num += (double)__ldg(p + ja);
+        else bad = true;
+        if (jb >= 0 && jb < len) den += (double)__ldg(p + jb);
+        else bad = true;
+      }
+    }
+  }
+  if (bad) flag_status(a.status, kStatusBadIndex);
+  for (int o = 16; o > 0; o >>= 1) {
+    num += __shfl_xor_sync(0xffffffffu, num, o);
+    den += __shfl_xor_sync(0xffffffffu, den, o);
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    s_num[warp] = num;
+    s_den[warp] = den;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double n = 0.0, d = 0.0;
+    for (int w = 0; w < kSimThreads / 32; ++w) {  // fixed order: deterministic
+      n += s_num[w];
+      d += s_den[w];
+    }
+    a.ratio[r] = d > 0.0 ? n / d : 0.0;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_similarity_rows(const SimArgs& a, int n_out, cudaStream_t st) {
+  if (n_out == 0) return cudaSuccess;
+  similarity_rows_kernel<<<n_out, kSimThreads, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+// Algorithm 1 with the readings of the DP bounds: layers 0..L-1, dp[0][0] = 0,
+// dp[0][j > 0] = -inf, dp[m][j] = max over i = m-1 .. j-1 of
+// dp[m-1][i] + sum_{l=i}^{j-1} S[i][l]; the answer is dp[M][L]; the smallest i
+// is kept among equal maxima; the anchors come back by backtracking.
+void select_anchors_dp(const double* S, int L, int M, int32_t* anchors, double* best) {
+  std::vector<double> cover((size_t)(L + 1) * (L + 1), 0.0);  // cover[i][j]
+  for (int i = 0; i < L; ++i) {
+    double run = 0.0;
+    for (int j = i + 1; j <= L; ++j) {
+      run += S[(size_t)i * L + (j - 1)];
+      cover[(size_t)i * (L + 1) + j] = run;
+    }
+  }
+  const double neg = -INFINITY;
+  std::vector<double> dp((size_t)(M + 1) * (L + 1), neg);
+  std::vector<int> arg((size_t)(M + 1) * (L + 1), -1);
+  auto at = [&](int m, int j) { return (size_t)m * (L + 1) + j; };
+  dp[at(0, 0)] = 0.0;
+  for (int m = 1; m <= M; ++m) {
+    for (int j = m; j <= L; ++j) {
+      double b = neg;
+      int bi = -1;
+      for (int i = m - 1; i < j; ++i) {
+        const double prev = dp[at(m - 1, i)];
+        if (prev == neg) continue;
+        const double v = prev + cover[(size_t)i * (L + 1) + j];
+        if (v > b) {
+          b = v;
+          bi = i;
+        }
+      }
+      dp[at(m, j)] = b;
+      arg[at(m, j)] = bi;
+    }
+  }
+  int j = L;
+  for (int m = M; m >= 1; --m) {
+    const int i = arg[at(m, j)];
+    anchors[m - 1] = i;  // backtracking visits the anchors from the last to the first
+    j = i;
+  }
+  *best = dp[at(M, L)];
+}
+
+}  // namespace kascade

@@ -72,4 +72,22 @@ size_t prefill_reuse_workspace_bytes(int B, int Hq, int Hkv, int N, int k_max);
 cudaError_t launch_prefill_anchor(const PrefillParams& p, cudaStream_t st);
 cudaError_t launch_prefill_reuse(const PrefillParams& p, cudaStream_t st);
 
+// ----------------------------------------------------------- calibration ----
+struct SimArgs {
+  const float* p_b;
+  int rows;
+  int64_t ld;
+  const int32_t* row_len;
+  const int32_t* row_k;
+  const int32_t* idx_a;
+  const int32_t* idx_b;
+  int k_max;
+  const int32_t* b_row;
+  const int32_t* a_row;
+  double* ratio;
+  unsigned* status;
+};
+cudaError_t launch_similarity_rows(const SimArgs& a, int n_out, cudaStream_t st);
+void select_anchors_dp(const double* S, int L, int M, int32_t* anchors, double* best);
+
 }  // namespace kascade
