@@ -343,6 +343,55 @@ def calibration_timing(dev, reps: int = 20):
             "head_remap_us": remap_us, "select_anchors_L32_M5_host_us": dp_us}
 
 
+def paged_timing(dec, reps: int = 20, page_size: int = 64):
+    """Paged-cache decode (outside the timed step): the workload's first anchor
+    layer and first reuse layer packed into 64-token pages in a seeded random
+    page order, timed against the contiguous calls on the same data."""
+    from long_context_emitting_b200 import api, paging, workload
+
+    cfg, sch, layers, maps, outs = dec
+    la = next(l for l in range(sch.n_layers) if sch.is_anchor(l))
+    lr = next((l for l in range(sch.n_layers) if not sch.is_anchor(l)), None)
+    if lr is None:
+        return None
+    sch.run_anchor(layers[la], outs[la])
+    sch.run_topk()
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(reps):
+            fn()
+        e.record()
+        torch.cuda.synchronize()
+        return s.elapsed_time(e) / reps * 1e3
+
+    res = {"page_size": page_size, "layout": "[num_pages, Hkv, page_size, 128], seeded random page order"}
+    ks, vs = workload.decode_cache_views(cfg, layers[la])
+    kp, vp, table, _ = paging.to_paged(ks, vs, page_size, seed=1)
+    out = torch.empty_like(outs[la])
+    lse = torch.empty_like(sch.lse)
+    pooled = torch.empty_like(sch.pooled)
+    ws = api.workspace(api.decode_anchor_workspace_bytes(cfg.B, cfg.Hq, cfg.Hkv, sch.max_T), kp.device)
+    res["anchor_us"] = timed(lambda: api.decode_anchor_paged(
+        layers[la]["q"], kp, vp, table, page_size, layers[la]["seq_len"], sch.max_T, sch.scale,
+        cfg.Hkv, out=out, lse=lse, pooled=pooled, ld_pooled=sch.ld, ws=ws))
+    res["anchor_contiguous_us"] = timed(lambda: sch.run_anchor(layers[la], outs[la]))
+    del kp, vp
+    ks, vs = workload.decode_cache_views(cfg, layers[lr])
+    kp, vp, table, _ = paging.to_paged(ks, vs, page_size, seed=2)
+    res["reuse_us"] = timed(lambda: api.decode_reuse_paged(
+        layers[lr]["q"], kp, vp, table, page_size, layers[lr]["seq_len"], sch.idx, sch.row_k,
+        maps[lr], sch.scale, cfg.Hkv, out=out, lse=lse))
+    res["reuse_contiguous_us"] = timed(lambda: sch.run_reuse(layers[lr], maps[lr], outs[lr]))
+    del kp, vp
+    torch.cuda.empty_cache()
+    return res
+
+
 def cpu_sample(steps: int = 1):
     """The float64 oracle on a bounded sample of the same workload (host cores).
 
@@ -649,6 +698,7 @@ def main():
 
     if dec and dist.rank == 0:
         out["calibration"] = calibration_timing(dev)
+        out["paged"] = paged_timing(dec)
     if not args.no_e2e:
         out["e2e"] = e2e(dec, pre, args, dist)
     if not args.no_cpu and dist.rank == 0:

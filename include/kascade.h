@@ -196,6 +196,33 @@ int kascade_prefill_reuse(kascade_shape s, int32_t N, const uint16_t* q, const u
                           float* lse, void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------- */
+/* Paged KV cache variants of the two decode calls (the explainer's serving
+ * integration keeps the cache in fixed-size pages).  Same operation, outputs
+ * and workspace (kascade_decode_{anchor,reuse}_workspace_bytes) as the
+ * contiguous calls; only where a token's K/V row lives differs:
+ *   k_pages, v_pages  device bf16 [num_pages, Hkv, page_size, 128], 16-byte aligned
+ *   block_table       device int32 [B, max_pages]: page j of sequence b holds its
+ *                     tokens j*page_size .. j*page_size + page_size - 1
+ *   page_size         multiple of 16 (>= 16)
+ * Host checks as for the contiguous calls, plus: num_pages >= 1, max_pages >= 1,
+ * and (anchor) max_pages * page_size >= max_T.  A block-table entry outside
+ * [0, num_pages) skips the tokens it holds and sets KASCADE_ERR_BAD_INDEX in the
+ * device status; a sequence longer than max_pages * page_size is skipped the same
+ * way.  Results are bit-identical to the contiguous calls on the same data. */
+int kascade_decode_anchor_paged(kascade_shape s, const uint16_t* q, const uint16_t* k_pages,
+                                const uint16_t* v_pages, int32_t num_pages,
+                                const int32_t* block_table, int32_t max_pages, int32_t page_size,
+                                const int32_t* seq_len, int32_t max_T, float scale, uint16_t* out,
+                                float* lse, float* pooled, int64_t ld_pooled, void* ws,
+                                size_t ws_bytes, void* stream);
+int kascade_decode_reuse_paged(kascade_shape s, const uint16_t* q, const uint16_t* k_pages,
+                               const uint16_t* v_pages, int32_t num_pages,
+                               const int32_t* block_table, int32_t max_pages, int32_t page_size,
+                               const int32_t* seq_len, const int32_t* idx, const int32_t* idx_k,
+                               int32_t k_max, const int32_t* head_map, float scale, uint16_t* out,
+                               float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------- */
 /* Calibration (Kascade explainer, レイヤー間類似度とアンカーレイヤー選択 and
  * 動的計画法): which layers are anchors and which anchor KV head each reuse
  * head follows are chosen offline from post-softmax distributions.

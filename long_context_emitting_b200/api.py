@@ -116,6 +116,59 @@ def decode_reuse(q, k, v, kv_off, seq_len, idx, idx_k, head_map, scale: float, H
     return out, lse
 
 
+# ------------------------------------------------------------ decode, paged ----
+def decode_anchor_paged(q, k_pages, v_pages, block_table, page_size: int, seq_len, max_T: int,
+                        scale: float, Hkv: int, out=None, lse=None, pooled=None,
+                        ld_pooled: Optional[int] = None, ws=None):
+    """kascade_decode_anchor over a paged cache (see paging.to_paged)."""
+    B, Hq, d = q.shape
+    _need_cuda("q", q, torch.bfloat16)
+    _need_cuda("k_pages", k_pages, torch.bfloat16)
+    _need_cuda("v_pages", v_pages, torch.bfloat16)
+    _need_cuda("block_table", block_table, torch.int32)
+    _need_cuda("seq_len", seq_len, torch.int32)
+    dev = q.device
+    if ld_pooled is None:
+        ld_pooled = (max_T + 3) // 4 * 4
+    out = torch.empty(B, Hq, d, dtype=torch.bfloat16, device=dev) if out is None else out
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=dev) if lse is None else lse
+    pooled = torch.empty(B, Hkv, ld_pooled, dtype=torch.float32, device=dev) if pooled is None else pooled
+    shape = Shape(B, Hq, Hkv, d)
+    need = _lib().kascade_decode_anchor_workspace_bytes(shape, max_T)
+    ws = workspace(need, dev) if ws is None else ws
+    rc = _lib().kascade_decode_anchor_paged(
+        shape, _ptr(q), _ptr(k_pages), _ptr(v_pages), int(k_pages.shape[0]), _ptr(block_table),
+        int(block_table.shape[1]), int(page_size), _ptr(seq_len), int(max_T), float(scale),
+        _ptr(out), _ptr(lse), _ptr(pooled), int(ld_pooled), _ptr(ws), ws.numel(), _stream())
+    check(rc, "kascade_decode_anchor_paged")
+    return out, lse, pooled
+
+
+def decode_reuse_paged(q, k_pages, v_pages, block_table, page_size: int, seq_len, idx, idx_k,
+                       head_map, scale: float, Hkv: int, out=None, lse=None, ws=None):
+    """kascade_decode_reuse over a paged cache (see paging.to_paged)."""
+    B, Hq, d = q.shape
+    for name, t, dt in (("q", q, torch.bfloat16), ("k_pages", k_pages, torch.bfloat16),
+                        ("v_pages", v_pages, torch.bfloat16), ("block_table", block_table, torch.int32),
+                        ("seq_len", seq_len, torch.int32), ("idx", idx, torch.int32),
+                        ("idx_k", idx_k, torch.int32), ("head_map", head_map, torch.int32)):
+        _need_cuda(name, t, dt)
+    k_max = idx.shape[-1]
+    dev = q.device
+    out = torch.empty(B, Hq, d, dtype=torch.bfloat16, device=dev) if out is None else out
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=dev) if lse is None else lse
+    shape = Shape(B, Hq, Hkv, d)
+    need = _lib().kascade_decode_reuse_workspace_bytes(shape, k_max)
+    ws = workspace(need, dev) if ws is None else ws
+    rc = _lib().kascade_decode_reuse_paged(
+        shape, _ptr(q), _ptr(k_pages), _ptr(v_pages), int(k_pages.shape[0]), _ptr(block_table),
+        int(block_table.shape[1]), int(page_size), _ptr(seq_len), _ptr(idx), _ptr(idx_k),
+        int(k_max), _ptr(head_map), float(scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+        _stream())
+    check(rc, "kascade_decode_reuse_paged")
+    return out, lse
+
+
 # ------------------------------------------------------------------ topk ----
 def topk(scores, row_len, row_k, k_max: int, out=None):
     """Row-wise Top-k (ties to lower index, ascending output; tail = -1)."""

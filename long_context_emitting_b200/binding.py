@@ -38,6 +38,8 @@ EXPORTS = (
     "kascade_prefill_anchor",
     "kascade_prefill_reuse_workspace_bytes",
     "kascade_prefill_reuse",
+    "kascade_decode_anchor_paged",
+    "kascade_decode_reuse_paged",
     "kascade_similarity_rows",
     "kascade_select_anchors",
     "kascade_get_device_status",
@@ -80,6 +82,10 @@ _SIGNATURES = {
     "kascade_prefill_reuse_workspace_bytes": (_SZ, [Shape, _I32, _I32]),
     "kascade_prefill_reuse": (ctypes.c_int, [Shape, _I32, _P, _P, _P, _P, _P, _I32, _P, _F, _P, _P,
                                              _P, _SZ, _P]),
+    "kascade_decode_anchor_paged": (ctypes.c_int, [Shape, _P, _P, _P, _I32, _P, _I32, _I32, _P, _I32,
+                                                   _F, _P, _P, _P, _I64, _P, _SZ, _P]),
+    "kascade_decode_reuse_paged": (ctypes.c_int, [Shape, _P, _P, _P, _I32, _P, _I32, _I32, _P, _P,
+                                                  _P, _I32, _P, _F, _P, _P, _P, _SZ, _P]),
     "kascade_similarity_rows": (ctypes.c_int, [_P, _I32, _I64, _P, _P, _P, _P, _I32, _I32, _P, _P,
                                                _P, _P]),
     "kascade_select_anchors": (ctypes.c_int, [_P, _I32, _I32, _P, _P]),

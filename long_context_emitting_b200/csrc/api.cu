@@ -144,6 +144,80 @@ int kascade_decode_reuse(kascade_shape s, const uint16_t* q, const uint16_t* k,
   return from_cuda(launch_decode_reuse(p, static_cast<cudaStream_t>(stream)));
 }
 
+// ------------------------------------------------------------ decode, paged --
+static int check_pages(const uint16_t* k, const uint16_t* v, const int32_t* block_table,
+                       int32_t num_pages, int32_t max_pages, int32_t page_size) {
+  if (!k || !v || !block_table || num_pages < 1 || max_pages < 1 || page_size < 16 ||
+      (page_size % 16))
+    return KASCADE_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || ((uintptr_t)block_table & 3)) return KASCADE_ERR_INVALID_ARG;
+  return KASCADE_OK;
+}
+
+int kascade_decode_anchor_paged(kascade_shape s, const uint16_t* q, const uint16_t* k_pages,
+                                const uint16_t* v_pages, int32_t num_pages,
+                                const int32_t* block_table, int32_t max_pages, int32_t page_size,
+                                const int32_t* seq_len, int32_t max_T, float scale, uint16_t* out,
+                                float* lse, float* pooled, int64_t ld_pooled, void* ws,
+                                size_t ws_bytes, void* stream) {
+  int rc = check_shape(s);
+  if (rc) return rc;
+  if (max_T < 0 || ld_pooled < max_T || (ld_pooled & 3) || !std::isfinite(scale))
+    return KASCADE_ERR_INVALID_ARG;
+  if (s.B == 0) return KASCADE_OK;
+  if ((rc = check_pages(k_pages, v_pages, block_table, num_pages, max_pages, page_size))) return rc;
+  if ((int64_t)max_pages * page_size < max_T) return KASCADE_ERR_INVALID_ARG;
+  if (!q || !seq_len || !out || !pooled || !ws) return KASCADE_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(pooled) || !aligned16(ws) ||
+      (lse && !aligned16(lse)) || ((uintptr_t)seq_len & 3))
+    return KASCADE_ERR_INVALID_ARG;
+  if (ws_bytes < kascade_decode_anchor_workspace_bytes(s, max_T)) return KASCADE_ERR_WORKSPACE_TOO_SMALL;
+  DecodeParams p = {};
+  p.B = s.B; p.Hq = s.Hq; p.Hkv = s.Hkv; p.G = s.Hq / s.Hkv;
+  p.q = q; p.k = k_pages; p.v = v_pages; p.seq_len = seq_len; p.max_T = max_T;
+  p.block_table = block_table; p.max_pages = max_pages; p.page_size = page_size;
+  p.num_pages = num_pages;
+  p.scale = scale; p.out = out; p.lse = lse; p.pooled = pooled; p.ld_pooled = ld_pooled;
+  p.ws = ws;
+  p.status = device_status_ptr();
+  if (!p.status) return KASCADE_ERR_CUDA;
+  return from_cuda(launch_decode_anchor(p, static_cast<cudaStream_t>(stream)));
+}
+
+int kascade_decode_reuse_paged(kascade_shape s, const uint16_t* q, const uint16_t* k_pages,
+                               const uint16_t* v_pages, int32_t num_pages,
+                               const int32_t* block_table, int32_t max_pages, int32_t page_size,
+                               const int32_t* seq_len, const int32_t* idx, const int32_t* idx_k,
+                               int32_t k_max, const int32_t* head_map, float scale, uint16_t* out,
+                               float* lse, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_shape(s);
+  if (rc) return rc;
+  if (k_max < 0 || !std::isfinite(scale)) return KASCADE_ERR_INVALID_ARG;
+  if (s.B == 0) return KASCADE_OK;
+  if ((rc = check_pages(k_pages, v_pages, block_table, num_pages, max_pages, page_size))) return rc;
+  const size_t need = kascade_decode_reuse_workspace_bytes(s, k_max);
+  if (!q || !seq_len || !idx || !idx_k || !head_map || !out || (need && !ws))
+    return KASCADE_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(out) || (ws && !aligned16(ws)) || (lse && !aligned16(lse)) ||
+      ((uintptr_t)seq_len & 3) || ((uintptr_t)idx & 3) || ((uintptr_t)idx_k & 3) ||
+      ((uintptr_t)head_map & 3))
+    return KASCADE_ERR_INVALID_ARG;
+  if (ws_bytes < need) return KASCADE_ERR_WORKSPACE_TOO_SMALL;
+  DecodeParams p = {};
+  p.B = s.B; p.Hq = s.Hq; p.Hkv = s.Hkv; p.G = s.Hq / s.Hkv;
+  p.q = q; p.k = k_pages; p.v = v_pages; p.seq_len = seq_len;
+  p.block_table = block_table; p.max_pages = max_pages; p.page_size = page_size;
+  p.num_pages = num_pages;
+  // a sequence longer than its block table's pages is flagged and skipped
+  const int64_t cap = (int64_t)max_pages * page_size;
+  p.max_T = cap > 0x7fffffff ? 0x7fffffff : (int)cap;
+  p.idx = idx; p.idx_k = idx_k; p.head_map = head_map; p.k_max = k_max;
+  p.scale = scale; p.out = out; p.lse = lse; p.ws = ws;
+  p.status = device_status_ptr();
+  if (!p.status) return KASCADE_ERR_CUDA;
+  return from_cuda(launch_decode_reuse(p, static_cast<cudaStream_t>(stream)));
+}
+
 // -------------------------------------------------------------------- topk --
 size_t kascade_topk_workspace_bytes(int32_t rows, int64_t ld) {
   (void)rows;

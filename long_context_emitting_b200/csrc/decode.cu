@@ -45,7 +45,9 @@ struct SplitArgs {
   const uint16_t* q;
   const uint16_t* k;
   const uint16_t* v;
-  const int64_t* kv_off;
+  const int64_t* kv_off;      // contiguous cache: sequence offsets (NULL when paged)
+  const int32_t* block_table; // paged cache: [B, max_pages] page of each page_size tokens
+  int max_pages, page_size, num_pages;
   const int32_t* seq_len;
   const int32_t* idx;
   const int32_t* idx_k;
@@ -69,7 +71,7 @@ template <bool GATHER>
 __device__ __forceinline__ int resolve_rows(const SplitArgs& a, int b, int h, int& T,
                                             int64_t& off, const int32_t*& rows) {
   T = a.seq_len[b];
-  off = a.kv_off[b];
+  off = a.block_table ? 0 : a.kv_off[b];
   bool ok = (T >= 0) && (T <= a.max_T) && ((off & 7) == 0) && off >= 0;
   int n = T;
   rows = nullptr;
@@ -97,6 +99,16 @@ struct Blk {
   int ia, ib;        // item positions (for the logits store)
   bool oka, okb;     // rows present
 };
+
+// Paged cache: element offset of token t of KV head h of sequence b in a
+// [num_pages, Hkv, page_size, 128] page store, or -1 when its page entry is out
+// of range.
+__device__ __forceinline__ int64_t paged_row(const SplitArgs& a, int b, int h, int t) {
+  const int pi = t / a.page_size;
+  const int page = __ldg(a.block_table + (int64_t)b * a.max_pages + pi);
+  if (page < 0 || page >= a.num_pages) return -1;
+  return (((int64_t)page * a.Hkv + h) * a.page_size + (t - pi * a.page_size)) * kHeadDim;
+}
 
 // Loads one 16-row block of the anchor's contiguous K/V stream into registers.
 __device__ __forceinline__ void load_blk(Blk& x, int i0, int i_end, const uint16_t* Kb, const uint16_t* Vb,
@@ -191,8 +203,11 @@ __device__ __forceinline__ void compute_blk(const Blk& x, WarpState& w, const ui
   }
 }
 
-// Decode anchor over the contiguous K/V stream: two register buffers (the
-// next block's loads in flight during the current block's math), 2 CTAs per SM.
+// Decode anchor over the K/V stream: two register buffers (the next block's
+// loads in flight during the current block's math), 2 CTAs per SM.  PAGED: a
+// warp's 16-token blocks start at multiples of 16 and the page size is a
+// multiple of 16, so each block lies in one page, looked up once per block.
+template <bool PAGED>
 __global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const SplitArgs a) {
   __shared__ float sm_o[kWarps][8][kHeadDim];
   __shared__ float sm_m[kWarps][8];
@@ -236,14 +251,32 @@ __global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const SplitAr
 
   float* lrow = a.logits + ((int64_t)b * a.Hkv + h) * a.max_T * G;
 
+  // the block of tokens i0 .. i0+15: contiguous, or through the block table
+  // (a bad page entry masks the whole block, read from page 0)
+  auto load = [&](Blk& x, int i0) {
+    if constexpr (PAGED) {
+      int64_t o = paged_row(a, b, h, i0);
+      int end = i_end;
+      if (o < 0) {
+        flag_status(a.status, kStatusBadIndex);
+        o = 0;
+        end = i0;
+      }
+      load_blk(x, 0, end - i0, a.k + o, a.v + o, gid, tig);
+      x.ia += i0;
+      x.ib += i0;
+    } else {
+      load_blk(x, i0, i_end, Kb, Vb, gid, tig);
+    }
+  };
   Blk x0, x1;
-  if (i_begin < i_end) load_blk(x0, i_begin, i_end, Kb, Vb, gid, tig);
+  if (i_begin < i_end) load(x0, i_begin);
   for (int i0 = i_begin; i0 < i_end; i0 += 32) {
     const bool has1 = i0 + 16 < i_end;
-    if (has1) load_blk(x1, i0 + 16, i_end, Kb, Vb, gid, tig);
+    if (has1) load(x1, i0 + 16);
     compute_blk<false>(x0, ws, qf, a.scale_log2, lrow, G, tig);
     if (!has1) break;
-    if (i0 + 32 < i_end) load_blk(x0, i0 + 32, i_end, Kb, Vb, gid, tig);
+    if (i0 + 32 < i_end) load(x0, i0 + 32);
     compute_blk<false>(x1, ws, qf, a.scale_log2, lrow, G, tig);
   }
 
@@ -313,6 +346,7 @@ __device__ __forceinline__ uint32_t gswz(int r, int c) {
   return (uint32_t)r * 256u + ((uint32_t)(c ^ ((r & 1) << 2)) << 4);
 }
 
+template <bool PAGED>
 __global__ void __launch_bounds__(kThreads, 3) decode_gather_kernel(const SplitArgs a) {
   extern __shared__ uint8_t gsm_raw[];
   uint8_t* gsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gsm_raw) + 127) & ~uintptr_t(127));
@@ -359,9 +393,17 @@ __global__ void __launch_bounds__(kThreads, 3) decode_gather_kernel(const SplitA
     // validity of the block's 16 rows (lanes 0..15), kept for the softmax mask
     const int itv = i_begin + 16 * bi + (lane & 15);
     bool okv = false;
+    int64_t rowv = 0;  // paged: element offset of row lane & 15 in the page store
     if (itv < i_end) {
       const int key = __ldg(rows + itv);
       okv = key >= 0 && key < T;
+      if constexpr (PAGED) {
+        if (okv) {
+          rowv = paged_row(a, b, h, key);
+          okv = rowv >= 0;
+          if (!okv) rowv = 0;
+        }
+      }
       if (!okv && lane < 16) flag_status(a.status, kStatusBadIndex);
     }
     const unsigned m = __ballot_sync(0xffffffffu, okv) & 0xffffu;
@@ -369,13 +411,20 @@ __global__ void __launch_bounds__(kThreads, 3) decode_gather_kernel(const SplitA
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int r = 2 * i + rpar;
-      const int it = i_begin + 16 * bi + r;
-      int key = it < i_end ? __ldg(rows + it) : 0;
       const bool ok = (m >> r) & 1u;
-      if (!ok) key = 0;  // zero-filled from a valid address (T >= 1 whenever there are items)
       const uint32_t o = gswz(r, c16);
-      cp_async16(dst + o, Kb + (int64_t)key * kHeadDim + c16 * 8, ok ? 16u : 0u);
-      cp_async16(dst + 4096u + o, Vb + (int64_t)key * kHeadDim + c16 * 8, ok ? 16u : 0u);
+      if constexpr (PAGED) {
+        int64_t ro = __shfl_sync(0xffffffffu, rowv, r);  // offset computed by lane r
+        if (!ok) ro = 0;  // zero-filled from a valid address (page 0)
+        cp_async16(dst + o, a.k + ro + c16 * 8, ok ? 16u : 0u);
+        cp_async16(dst + 4096u + o, a.v + ro + c16 * 8, ok ? 16u : 0u);
+      } else {
+        const int it = i_begin + 16 * bi + r;
+        int key = it < i_end ? __ldg(rows + it) : 0;
+        if (!ok) key = 0;  // zero-filled from a valid address (T >= 1 whenever there are items)
+        cp_async16(dst + o, Kb + (int64_t)key * kHeadDim + c16 * 8, ok ? 16u : 0u);
+        cp_async16(dst + 4096u + o, Vb + (int64_t)key * kHeadDim + c16 * 8, ok ? 16u : 0u);
+      }
     }
   };
 
@@ -547,7 +596,7 @@ __global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(const C
 
   if (a.logits) {
     int T = a.seq_len[b];
-    const int64_t off = a.kv_off[b];
+    const int64_t off = a.kv_off ? a.kv_off[b] : 0;  // NULL for a paged cache
     if (T < 0 || T > a.max_T || (off & 7) || off < 0) T = 0;
     const int t_lo = chunk * kPoolChunk;
     const int t_hi = min(t_lo + kPoolChunk, T);
@@ -625,7 +674,11 @@ DecodeSplit decode_split_for(int units, int n_items, bool gather) {
     return s;
   }
   // Largest per-warp run (<= KASCADE_DECODE_MAX_TPW items) that still gives at
-  // least KASCADE_DECODE_TARGET_CTAS CTAs.
+  // least KASCADE_DECODE_TARGET_CTAS CTAs.  Runs stay multiples of 16 (halving
+  // from a power of two >= 16), which the paged path relies on: a 16-token block
+  // never crosses a page.
+  static_assert(KASCADE_DECODE_MAX_TPW >= 16 && (KASCADE_DECODE_MAX_TPW & (KASCADE_DECODE_MAX_TPW - 1)) == 0,
+                "per-warp runs must stay multiples of 16");
   constexpr int kTargetCtas = KASCADE_DECODE_TARGET_CTAS;
   int tpw = KASCADE_DECODE_MAX_TPW;
   while (tpw > 16) {
@@ -652,6 +705,9 @@ static cudaError_t launch_decode(const DecodeParams& p, bool gather, cudaStream_
 
   SplitArgs a;
   a.q = p.q; a.k = p.k; a.v = p.v; a.kv_off = p.kv_off; a.seq_len = p.seq_len;
+  a.block_table = p.block_table; a.max_pages = p.max_pages; a.page_size = p.page_size;
+  a.num_pages = p.num_pages;
+  const bool paged = p.block_table != nullptr;
   a.idx = p.idx; a.idx_k = p.idx_k; a.head_map = p.head_map; a.k_max = p.k_max;
   a.Hq = p.Hq; a.Hkv = p.Hkv; a.G = p.G; a.max_T = p.max_T;
   a.tok_per_warp = sp.tok_per_warp;
@@ -667,7 +723,8 @@ static cudaError_t launch_decode(const DecodeParams& p, bool gather, cudaStream_
   dim3 grid(sp.nsplit, p.Hkv, p.B);
   if (gather) {
     // reuse: the nsplit CTAs of each (b, h) are one cluster and merge on chip
-    cudaError_t e = cudaFuncSetAttribute(decode_gather_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGSmem);
+    auto kern = paged ? decode_gather_kernel<true> : decode_gather_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGSmem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
@@ -681,11 +738,12 @@ static cudaError_t launch_decode(const DecodeParams& p, bool gather, cudaStream_
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, decode_gather_kernel, a);
+    e = cudaLaunchKernelEx(&cfg, kern, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }
-  decode_split_kernel<<<grid, kThreads, 0, st>>>(a);
+  if (paged) decode_split_kernel<true><<<grid, kThreads, 0, st>>>(a);
+  else decode_split_kernel<false><<<grid, kThreads, 0, st>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 

@@ -16,7 +16,9 @@ struct DecodeParams {
   const uint16_t* q;
   const uint16_t* k;
   const uint16_t* v;
-  const int64_t* kv_off;
+  const int64_t* kv_off;        // contiguous cache (NULL when paged)
+  const int32_t* block_table;   // paged cache [B, max_pages] (NULL when contiguous)
+  int max_pages = 0, page_size = 0, num_pages = 0;
   const int32_t* seq_len;
   int max_T;
   // gather (reuse) only
