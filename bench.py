@@ -392,6 +392,43 @@ def paged_timing(dec, reps: int = 20, page_size: int = 64):
     return res
 
 
+def long_context_timing(dev, T: int = 524288, reps: int = 10):
+    """A 512K-token decode (B = 1, the longest context of the evaluation's
+    latency table), outside the timed step: anchor, Top-k and one reuse layer."""
+    from long_context_emitting_b200 import workload
+    from long_context_emitting_b200.schedule import DecodeSchedule
+
+    cfg = workload.scaled(workload.DECODE_4K, name=f"decode_b1_t{T}", B=1, T=T, n_layers=2)
+    sch = DecodeSchedule(cfg.B, cfg.Hq, cfg.Hkv, cfg.seq_lens(), (0,), 2, dev)
+    la, lr = workload.decode_layer(cfg, 0, dev), workload.decode_layer(cfg, 1, dev)
+    hm = workload.head_map(cfg, 1).to(dev)
+    out = torch.empty(cfg.B, cfg.Hq, cfg.d, dtype=torch.bfloat16, device=dev)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(reps):
+            fn()
+        e.record()
+        torch.cuda.synchronize()
+        return s.elapsed_time(e) / reps * 1e3
+
+    anchor_us = timed(lambda: sch.run_anchor(la, out))
+    topk_us = timed(sch.run_topk)
+    reuse_us = timed(lambda: sch.run_reuse(lr, hm, out))
+    kv = T * cfg.Hkv * (cfg.d * 2 * 2 + 4)
+    gathered = cfg.Hkv * sch.k_max * cfg.d * 2 * 2
+    res = {"workload": cfg.name, "k": int(sch.k_max), "anchor_us": anchor_us,
+           "anchor_hbm_gbs": kv / (anchor_us * 1e-6) / 1e9, "topk_us": topk_us,
+           "reuse_us": reuse_us, "reuse_hbm_gbs": gathered / (reuse_us * 1e-6) / 1e9}
+    del la, lr, sch
+    torch.cuda.empty_cache()
+    return res
+
+
 def cpu_sample(steps: int = 1):
     """The float64 oracle on a bounded sample of the same workload (host cores).
 
@@ -699,6 +736,7 @@ def main():
     if dec and dist.rank == 0:
         out["calibration"] = calibration_timing(dev)
         out["paged"] = paged_timing(dec)
+        out["long_context"] = long_context_timing(dev)
     if not args.no_e2e:
         out["e2e"] = e2e(dec, pre, args, dist)
     if not args.no_cpu and dist.rank == 0:

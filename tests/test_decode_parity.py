@@ -87,6 +87,13 @@ def test_decode_small_ragged():
     _check_layer_pair(cfg)
 
 
+def test_decode_b1_t262144():
+    # a 256K context (rows longer than the Top-k kernel's shared-memory cache are
+    # re-read from L2 on every radix pass)
+    cfg = workload.scaled(workload.DECODE_4K, name="decode_b1_t262144", B=1, T=262144)
+    _check_layer_pair(cfg)
+
+
 @pytest.mark.parametrize("Hq,Hkv", [(8, 8), (16, 8), (64, 8)])
 def test_decode_gqa_group_sizes(Hq, Hkv):
     # G = 1, 2 and 8 query heads per KV head (padding rows of the mma tile for G < 8)

@@ -101,6 +101,11 @@ def test_prefill_n65536_sampled_tiles():
     _check(workload.PREFILL_64K, tiles=[0, 2, 300, 511])
 
 
+def test_prefill_n131072_sampled_tiles():
+    cfg = workload.scaled(workload.PREFILL_64K, name="prefill_b1_n131072", N=131072)
+    _check(cfg, tiles=[0, 3, 1023])
+
+
 def test_prefill_reuse_full_prefix_is_dense():
     cfg = workload.scaled(workload.PREFILL_16K, name="prefill_dense_eq", N=512)
     inp = workload.prefill_layer(cfg, 0, DEV)

@@ -61,7 +61,7 @@ def test_topk_ragged_rows_and_short_rows():
     _check(scores, lens, ks, k_max=max(ks) + 3)
 
 
-@pytest.mark.parametrize("n,rows", [(32768, 3), (49152, 2), (49153, 2), (65536, 2), (131072, 2)])
+@pytest.mark.parametrize("n,rows", [(32768, 3), (49152, 2), (49153, 2), (65536, 2), (131072, 2), (524288, 2)])
 def test_topk_long_rows_cached_and_streamed(n, rows):
     # rows beyond 49152 keys are re-read from global memory on every pass;
     # the row stride is padded to a multiple of 4 floats (16-byte rows)
