@@ -663,10 +663,12 @@ DecodeSplit decode_split_for(int units, int n_items, bool gather) {
   DecodeSplit s;
   if (gather) {
     // One wave of the gather kernel (3 resident CTAs per SM): split each row
-    // into floor(444 / rows) CTAs (between 1 and 8), 4 warps each, 16-row blocks.
+    // into floor(444 / rows) CTAs (between 1 and 16), 4 warps each, 16-row
+    // blocks.  The splits of a row form one thread-block cluster: up to 8 is the
+    // portable size, 16 needs the non-portable attribute set at launch.
     constexpr int kSlots = 3 * 148;
     int nsplit = units >= kSlots ? 1 : kSlots / units;
-    if (nsplit > 8) nsplit = 8;  // the splits of a row form one (portable-size) cluster
+    if (nsplit > 16) nsplit = 16;
     int tpw = (n_items + 4 * nsplit - 1) / (4 * nsplit);
     tpw = ((tpw + 15) / 16) * 16;
     s.tok_per_warp = tpw > 16 ? tpw : 16;
@@ -726,6 +728,10 @@ static cudaError_t launch_decode(const DecodeParams& p, bool gather, cudaStream_
     auto kern = paged ? decode_gather_kernel<true> : decode_gather_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGSmem);
     if (e != cudaSuccess) return e;
+    if (sp.nsplit > 8) {
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e != cudaSuccess) return e;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = dim3(kThreads);
