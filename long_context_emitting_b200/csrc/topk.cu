@@ -4,6 +4,13 @@
 // (exact Top-k of the post-softmax distribution in anchor layers, one set per
 // key head per ヘッドリマッピング) with k from › Top-k設定.
 //
+// Rows longer than the shared-memory cache run on topk_cluster_kernel: one
+// thread-block cluster of C CTAs per row (C a power of two up to 16), each CTA
+// caching one slice of the row.  Every radix pass sums the CTAs' histograms
+// through distributed shared memory (each CTA computes the same selection), and
+// the compaction takes each CTA's output offsets from the counts of the
+// lower-ranked CTAs, so the result is the single-CTA kernel's, bit for bit.
+//
 // One CTA of 1024 threads per row.  Scores are mapped to order-preserving
 // unsigned keys (-0.0 folded onto +0.0), cached in shared memory when the row
 // fits (otherwise re-read from global memory / L2 on every pass), and an
@@ -13,6 +20,8 @@
 // yields ascending indices with the lower-index tie-break.
 #include "common.cuh"
 #include "internal.h"
+
+#include <cooperative_groups.h>
 
 namespace kascade {
 
@@ -198,6 +207,152 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkArgs a) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Long rows: one cluster of C CTAs per row.  All control flow that reaches a
+// cluster barrier depends only on the row (its length, k, status), which every
+// CTA of the cluster reads alike, so the CTAs always meet at every barrier.
+__global__ void __launch_bounds__(kThreads, 1) topk_cluster_kernel(const TopkArgs a, int C, int seg) {
+  namespace cg = cooperative_groups;
+  extern __shared__ uint32_t smem[];
+  uint32_t* hist = smem;                 // kBins (this CTA's slice)
+  uint32_t* scratch = smem + kBins;      // 64 words
+  uint32_t* keys = smem + kBins + 64;    // seg keys
+  __shared__ int s_sel_bin, s_sel_above;
+  __shared__ uint32_t s_wgt[kWarpsPerRow], s_weq[kWarpsPerRow];
+  __shared__ uint32_t s_cta_gt, s_cta_eq;
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int row = blockIdx.x / C;
+  const int tid = threadIdx.x;
+  const int len = a.row_len[row];
+  const int k = a.row_k[row];
+  int32_t* out = a.idx_out + (int64_t)row * a.k_max;
+  const float* src = a.scores + (int64_t)row * a.ld;
+
+  if (len < 0 || (int64_t)len > a.ld || k < 0 || k > len || k > a.k_max) {
+    if (rank == 0) {
+      if (tid == 0) flag_status(a.status, kStatusBadIndex);
+      for (int i = tid; i < a.k_max; i += kThreads) out[i] = -1;
+    }
+    return;  // every CTA of the cluster takes this branch
+  }
+  if (rank == 0)
+    for (int i = k + tid; i < a.k_max; i += kThreads) out[i] = -1;
+
+  // this CTA's slice [lo, hi) of the row, cached as order-preserving keys
+  const int lo = min(rank * seg, len), hi = min(lo + seg, len);
+  const int n = hi - lo;
+  {
+    int nan_seen = 0;
+    const uint32_t* bits = reinterpret_cast<const uint32_t*>(src) + lo;
+    for (int i = tid; i < n; i += kThreads) {
+      const uint32_t f = __ldg(bits + i);
+      nan_seen |= is_nan_bits(f);
+      keys[i] = order_key(f);
+    }
+    if (__syncthreads_or(nan_seen) && tid == 0) flag_status(a.status, kStatusNonFinite);
+  }
+  if (k == 0) return;
+  if (k == len) {
+    for (int i = tid; i < n; i += kThreads) out[lo + i] = lo + i;
+    return;
+  }
+
+  // ---- radix select over the whole row: 11 / 11 / 10 bits --------------------
+  uint32_t prefix = 0u, pmask = 0u;
+  int k_rem = k;
+#pragma unroll 1
+  for (int pass = 0; pass < 3; ++pass) {
+    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+    const uint32_t dmask = pass < 2 ? 0x7ffu : 0x3ffu;
+    for (int i = tid; i < kBins; i += kThreads) hist[i] = 0u;
+    __syncthreads();
+    for (int i = tid; i < n; i += kThreads) {
+      const uint32_t key = keys[i];
+      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1u);
+    }
+    cluster.sync();  // every CTA's histogram is complete
+    // thread t owns bins hi = 2047-2t and lo = 2046-2t, summed over the cluster
+    uint32_t c_hi = 0u, c_lo = 0u;
+    for (int r = 0; r < C; ++r) {
+      const uint32_t* h = cluster.map_shared_rank(hist, r);
+      c_hi += h[kBins - 1 - 2 * tid];
+      c_lo += h[kBins - 2 - 2 * tid];
+    }
+    const uint32_t incl = block_inclusive_scan(c_hi + c_lo, scratch);
+    const uint32_t excl = incl - c_hi - c_lo;
+    const uint32_t kr = (uint32_t)k_rem;
+    if (excl < kr && kr <= excl + c_hi) {
+      s_sel_bin = kBins - 1 - 2 * tid;
+      s_sel_above = (int)excl;
+    } else if (excl + c_hi < kr && kr <= incl) {
+      s_sel_bin = kBins - 2 - 2 * tid;
+      s_sel_above = (int)(excl + c_hi);
+    }
+    cluster.sync();  // every CTA has read every histogram before the next pass clears its own
+    k_rem -= s_sel_above;
+    prefix |= (uint32_t)s_sel_bin << shift;
+    pmask |= dmask << shift;
+  }
+  const uint32_t tau = prefix;
+  const int need_eq = k_rem;
+
+  // ---- ordered compaction across the cluster ---------------------------------
+  const int lane = tid & 31, warp = tid >> 5;
+  const int wseg = (((n + kWarpsPerRow - 1) / kWarpsPerRow) + 31) & ~31;
+  const int s_lo = min(warp * wseg, n), s_hi = min(s_lo + wseg, n);
+  uint32_t n_gt = 0, n_eq = 0;
+  for (int base = s_lo; base < s_hi; base += 32) {
+    const int i = base + lane;
+    const uint32_t key = i < s_hi ? keys[i] : 0u;
+    n_gt += __popc(__ballot_sync(0xffffffffu, i < s_hi && key > tau));
+    n_eq += __popc(__ballot_sync(0xffffffffu, i < s_hi && key == tau));
+  }
+  if (lane == 0) {
+    s_wgt[warp] = n_gt;
+    s_weq[warp] = n_eq;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    uint32_t g = 0, e = 0;
+    for (int w = 0; w < kWarpsPerRow; ++w) {
+      g += s_wgt[w];
+      e += s_weq[w];
+    }
+    s_cta_gt = g;
+    s_cta_eq = e;
+  }
+  cluster.sync();  // every CTA's counts are published
+  uint32_t gt_before = 0, eq_before = 0;
+  for (int r = 0; r < rank; ++r) {
+    gt_before += *cluster.map_shared_rank(&s_cta_gt, r);
+    eq_before += *cluster.map_shared_rank(&s_cta_eq, r);
+  }
+  for (int w = 0; w < warp; ++w) {
+    gt_before += s_wgt[w];
+    eq_before += s_weq[w];
+  }
+  cluster.sync();  // the peers' counts have been read before any CTA exits
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  for (int base = s_lo; base < s_hi; base += 32) {
+    const int i = base + lane;
+    const uint32_t key = i < s_hi ? keys[i] : 0u;
+    const bool is_gt = i < s_hi && key > tau;
+    const bool is_eq = i < s_hi && key == tau;
+    const uint32_t mg = __ballot_sync(0xffffffffu, is_gt);
+    const uint32_t me = __ballot_sync(0xffffffffu, is_eq);
+    const uint32_t my_gt = gt_before + __popc(mg & lt_mask);
+    const uint32_t my_eq = eq_before + __popc(me & lt_mask);
+    if (is_gt || (is_eq && my_eq < (uint32_t)need_eq)) {
+      const uint32_t pos = my_gt + min(my_eq, (uint32_t)need_eq);
+      out[pos] = lo + i;
+    }
+    gt_before += __popc(mg);
+    eq_before += __popc(me);
+  }
+}
+
 }  // namespace
 
 size_t topk_smem_bytes(int64_t ld) {
@@ -218,6 +373,38 @@ cudaError_t launch_topk(const float* scores, int rows, int64_t ld, const int32_t
   a.idx_out = idx_out;
   a.cache_cap = (int)(ld < kCacheMaxKeys ? ld : kCacheMaxKeys);
   a.status = status;
+  if (ld > kCacheMaxKeys) {
+    // one cluster of C CTAs per row, C the smallest power of two whose slices fit the cache
+    int C = 2;
+    while (C < 16 && (ld + C - 1) / C > kCacheMaxKeys) C *= 2;
+    int seg = (int)((ld + C - 1) / C);
+    seg = (seg + 31) & ~31;
+    if (seg <= kCacheMaxKeys) {
+      const size_t smem = (size_t)(kBins + 64 + seg) * sizeof(uint32_t);
+      cudaError_t e = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)topk_smem_bytes(kCacheMaxKeys));
+      if (e != cudaSuccess) return e;
+      if (C > 8) {
+        e = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+      }
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)(rows * C));
+      cfg.blockDim = dim3(kThreads);
+      cfg.dynamicSmemBytes = smem;
+      cfg.stream = st;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = (unsigned)C;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel, a, C, seg);
+      if (e != cudaSuccess) return e;
+      return cudaGetLastError();
+    }
+  }
   const size_t smem = topk_smem_bytes(ld);
   cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)topk_smem_bytes(kCacheMaxKeys));
