@@ -7,8 +7,10 @@ Modules:
   api       -- tensor-level calls of the same names on the current CUDA stream
   schedule  -- anchor / Top-k / reuse layer schedule with preallocated buffers
   workload  -- seeded synthetic inputs shaped like the evaluated workloads
+  paging    -- packing per-sequence K/V caches into a page store (paged decode)
+  replicas  -- per-rank workloads for multi-GPU replica runs
   build     -- nvcc build of libkascade.so for sm_100a
 """
-from . import api, binding, schedule, workload  # noqa: F401
+from . import api, binding, paging, schedule, workload  # noqa: F401
 
-__all__ = ["api", "binding", "schedule", "workload"]
+__all__ = ["api", "binding", "paging", "schedule", "workload"]
