@@ -429,6 +429,58 @@ def long_context_timing(dev, T: int = 524288, reps: int = 10):
     return res
 
 
+def f16_timing(dec, pre, reps: int = 10):
+    """The float16 entry points (the evaluation's precision) on the workloads'
+    first anchor and reuse layers converted to float16, outside the timed step,
+    next to the bfloat16 calls on the same layers."""
+    from long_context_emitting_b200 import api
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(reps):
+            fn()
+        e.record()
+        torch.cuda.synchronize()
+        return s.elapsed_time(e) / reps * 1e3
+
+    def half(inp):
+        return {n: (t.to(torch.float16) if n in ("q", "k", "v") else t) for n, t in inp.items()}
+
+    res = {}
+    if dec:
+        cfg, sch, layers, maps, outs = dec
+        la = next(l for l in range(sch.n_layers) if sch.is_anchor(l))
+        lr = next((l for l in range(sch.n_layers) if not sch.is_anchor(l)), None)
+        a16 = half(layers[la])
+        o16 = torch.empty(outs[la].shape, dtype=torch.float16, device=outs[la].device)
+        res["decode_anchor_us"] = timed(lambda: sch.run_anchor(a16, o16))
+        res["decode_anchor_bf16_us"] = timed(lambda: sch.run_anchor(layers[la], outs[la]))
+        sch.run_topk()
+        del a16
+        if lr is not None:
+            r16 = half(layers[lr])
+            res["decode_reuse_us"] = timed(lambda: sch.run_reuse(r16, maps[lr], o16))
+            res["decode_reuse_bf16_us"] = timed(lambda: sch.run_reuse(layers[lr], maps[lr], outs[lr]))
+            del r16
+    if pre:
+        cfg, sch, layers, maps, outs = pre
+        a16 = half(layers[0])
+        o16 = torch.empty_like(a16["q"])
+        res["prefill_anchor_ms"] = timed(lambda: sch.run_anchor(a16, o16)) / 1e3
+        res["prefill_anchor_bf16_ms"] = timed(lambda: sch.run_anchor(layers[0], outs[0])) / 1e3
+        sch.run_topk()
+        if sch.n_layers > 1:
+            r16 = half(layers[1])
+            res["prefill_reuse_ms"] = timed(lambda: sch.run_reuse(r16, maps[1], o16)) / 1e3
+            res["prefill_reuse_bf16_ms"] = timed(lambda: sch.run_reuse(layers[1], maps[1], outs[1])) / 1e3
+    torch.cuda.empty_cache()
+    return res
+
+
 def cpu_sample(steps: int = 1):
     """The float64 oracle on a bounded sample of the same workload (host cores).
 
@@ -737,6 +789,8 @@ def main():
         out["calibration"] = calibration_timing(dev)
         out["paged"] = paged_timing(dec)
         out["long_context"] = long_context_timing(dev)
+    if dist.rank == 0 and (dec or pre):
+        out["f16"] = f16_timing(dec, pre)
     if not args.no_e2e:
         out["e2e"] = e2e(dec, pre, args, dist)
     if not args.no_cpu and dist.rank == 0:

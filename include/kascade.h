@@ -196,6 +196,29 @@ int kascade_prefill_reuse(kascade_shape s, int32_t N, const uint16_t* q, const u
                           float* lse, void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------- */
+/* fp16 variants (the evaluation's precision): the same contracts as the four
+ * calls above, with q, k, v and out holding IEEE half-precision values (the
+ * same uint16_t bit containers) instead of bfloat16.  Accumulation, softmax,
+ * LSE and pooled probabilities stay fp32; workspace sizes are those of the
+ * bfloat16 calls. */
+int kascade_decode_anchor_f16(kascade_shape s, const uint16_t* q, const uint16_t* k,
+                              const uint16_t* v, const int64_t* kv_off, const int32_t* seq_len,
+                              int32_t max_T, float scale, uint16_t* out, float* lse, float* pooled,
+                              int64_t ld_pooled, void* ws, size_t ws_bytes, void* stream);
+int kascade_decode_reuse_f16(kascade_shape s, const uint16_t* q, const uint16_t* k,
+                             const uint16_t* v, const int64_t* kv_off, const int32_t* seq_len,
+                             const int32_t* idx, const int32_t* idx_k, int32_t k_max,
+                             const int32_t* head_map, float scale, uint16_t* out, float* lse,
+                             void* ws, size_t ws_bytes, void* stream);
+int kascade_prefill_anchor_f16(kascade_shape s, int32_t N, const uint16_t* q, const uint16_t* k,
+                               const uint16_t* v, float scale, uint16_t* out, float* lse,
+                               float* pooled, void* ws, size_t ws_bytes, void* stream);
+int kascade_prefill_reuse_f16(kascade_shape s, int32_t N, const uint16_t* q, const uint16_t* k,
+                              const uint16_t* v, const int32_t* idx, const int32_t* idx_k,
+                              int32_t k_max, const int32_t* head_map, float scale, uint16_t* out,
+                              float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------- */
 /* Paged KV cache variants of the two decode calls (the explainer's serving
  * integration keeps the cache in fixed-size pages).  Same operation, outputs
  * and workspace (kascade_decode_{anchor,reuse}_workspace_bytes) as the

@@ -36,6 +36,17 @@ def _need_cuda(name: str, t: torch.Tensor, dtype: torch.dtype) -> None:
         raise ValueError(f"{name} must be contiguous")
 
 
+_DATA_DTYPES = (torch.bfloat16, torch.float16)
+
+
+def _data_suffix(*ts) -> str:
+    """'' for bfloat16 q/k/v/out, '_f16' for float16 (all of one call alike)."""
+    dt = ts[0].dtype
+    if dt not in _DATA_DTYPES or any(t.dtype != dt for t in ts):
+        raise TypeError("q, k, v must all be bfloat16 or all float16")
+    return "_f16" if dt == torch.float16 else ""
+
+
 def _bits(t: torch.Tensor) -> torch.Tensor:
     return t.view(torch.int16) if t.dtype == torch.bfloat16 else t
 
@@ -65,26 +76,27 @@ def decode_anchor_workspace_bytes(B, Hq, Hkv, max_T) -> int:
 
 def decode_anchor(q, k, v, kv_off, seq_len, max_T: int, scale: float, Hkv: int,
                   out=None, lse=None, pooled=None, ld_pooled: Optional[int] = None, ws=None):
-    """Dense decode attention + GQA-pooled probabilities (kascade_decode_anchor)."""
+    """Dense decode attention + GQA-pooled probabilities (kascade_decode_anchor; the
+    _f16 entry point when q, k, v are float16)."""
     B, Hq, d = q.shape
-    _need_cuda("q", q, torch.bfloat16)
-    _need_cuda("k", k, torch.bfloat16)
-    _need_cuda("v", v, torch.bfloat16)
+    sfx = _data_suffix(q, k, v)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need_cuda(name, t, q.dtype)
     _need_cuda("kv_off", kv_off, torch.int64)
     _need_cuda("seq_len", seq_len, torch.int32)
     dev = q.device
     if ld_pooled is None:
         ld_pooled = (max_T + 3) // 4 * 4
-    out = torch.empty(B, Hq, d, dtype=torch.bfloat16, device=dev) if out is None else out
+    out = torch.empty(B, Hq, d, dtype=q.dtype, device=dev) if out is None else out
     lse = torch.empty(B, Hq, dtype=torch.float32, device=dev) if lse is None else lse
     pooled = torch.empty(B, Hkv, ld_pooled, dtype=torch.float32, device=dev) if pooled is None else pooled
     shape = Shape(B, Hq, Hkv, d)
     need = _lib().kascade_decode_anchor_workspace_bytes(shape, max_T)
     ws = workspace(need, dev) if ws is None else ws
-    rc = _lib().kascade_decode_anchor(shape, _ptr(q), _ptr(k), _ptr(v), _ptr(kv_off), _ptr(seq_len),
+    rc = getattr(_lib(), "kascade_decode_anchor" + sfx)(shape, _ptr(q), _ptr(k), _ptr(v), _ptr(kv_off), _ptr(seq_len),
                                       int(max_T), float(scale), _ptr(out), _ptr(lse), _ptr(pooled),
                                       int(ld_pooled), _ptr(ws), ws.numel(), _stream())
-    check(rc, "kascade_decode_anchor")
+    check(rc, "kascade_decode_anchor" + sfx)
     return out, lse, pooled
 
 
@@ -94,25 +106,27 @@ def decode_reuse_workspace_bytes(B, Hq, Hkv, k_max) -> int:
 
 def decode_reuse(q, k, v, kv_off, seq_len, idx, idx_k, head_map, scale: float, Hkv: int,
                  out=None, lse=None, ws=None):
-    """Sparse decode attention over anchor indices via a head map (kascade_decode_reuse)."""
+    """Sparse decode attention over anchor indices via a head map (kascade_decode_reuse;
+    the _f16 entry point when q, k, v are float16)."""
     B, Hq, d = q.shape
-    for name, t, dt in (("q", q, torch.bfloat16), ("k", k, torch.bfloat16), ("v", v, torch.bfloat16),
+    sfx = _data_suffix(q, k, v)
+    for name, t, dt in (("q", q, q.dtype), ("k", k, q.dtype), ("v", v, q.dtype),
                         ("kv_off", kv_off, torch.int64), ("seq_len", seq_len, torch.int32),
                         ("idx", idx, torch.int32), ("idx_k", idx_k, torch.int32),
                         ("head_map", head_map, torch.int32)):
         _need_cuda(name, t, dt)
     k_max = idx.shape[-1]
     dev = q.device
-    out = torch.empty(B, Hq, d, dtype=torch.bfloat16, device=dev) if out is None else out
+    out = torch.empty(B, Hq, d, dtype=q.dtype, device=dev) if out is None else out
     lse = torch.empty(B, Hq, dtype=torch.float32, device=dev) if lse is None else lse
     shape = Shape(B, Hq, Hkv, d)
     need = _lib().kascade_decode_reuse_workspace_bytes(shape, k_max)
     ws = workspace(need, dev) if ws is None else ws
-    rc = _lib().kascade_decode_reuse(shape, _ptr(q), _ptr(k), _ptr(v), _ptr(kv_off), _ptr(seq_len),
+    rc = getattr(_lib(), "kascade_decode_reuse" + sfx)(shape, _ptr(q), _ptr(k), _ptr(v), _ptr(kv_off), _ptr(seq_len),
                                      _ptr(idx), _ptr(idx_k), int(k_max), _ptr(head_map),
                                      float(scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
                                      _stream())
-    check(rc, "kascade_decode_reuse")
+    check(rc, "kascade_decode_reuse" + sfx)
     return out, lse
 
 
@@ -190,11 +204,13 @@ def prefill_anchor_workspace_bytes(B, Hq, Hkv, N) -> int:
 
 
 def prefill_anchor(q, k, v, scale: float, out=None, lse=None, pooled=None, ws=None):
-    """Dense causal prefill attention + tile-pooled probabilities (kascade_prefill_anchor)."""
+    """Dense causal prefill attention + tile-pooled probabilities (kascade_prefill_anchor;
+    the _f16 entry point when q, k, v are float16)."""
     B, Hq, N, d = q.shape
     Hkv = k.shape[1]
+    sfx = _data_suffix(q, k, v)
     for name, t in (("q", q), ("k", k), ("v", v)):
-        _need_cuda(name, t, torch.bfloat16)
+        _need_cuda(name, t, q.dtype)
     dev = q.device
     out = torch.empty_like(q) if out is None else out
     lse = torch.empty(B, Hq, N, dtype=torch.float32, device=dev) if lse is None else lse
@@ -203,10 +219,10 @@ def prefill_anchor(q, k, v, scale: float, out=None, lse=None, pooled=None, ws=No
     shape = Shape(B, Hq, Hkv, d)
     need = _lib().kascade_prefill_anchor_workspace_bytes(shape, N)
     ws = workspace(need, dev) if ws is None else ws
-    rc = _lib().kascade_prefill_anchor(shape, int(N), _ptr(q), _ptr(k), _ptr(v), float(scale),
+    rc = getattr(_lib(), "kascade_prefill_anchor" + sfx)(shape, int(N), _ptr(q), _ptr(k), _ptr(v), float(scale),
                                        _ptr(out), _ptr(lse), _ptr(pooled), _ptr(ws), ws.numel(),
                                        _stream())
-    check(rc, "kascade_prefill_anchor")
+    check(rc, "kascade_prefill_anchor" + sfx)
     return out, lse, pooled
 
 
@@ -215,10 +231,12 @@ def prefill_reuse_workspace_bytes(B, Hq, Hkv, N, k_max) -> int:
 
 
 def prefill_reuse(q, k, v, idx, idx_k, head_map, scale: float, out=None, lse=None, ws=None):
-    """Sparse causal prefill attention over tile indices + diagonal (kascade_prefill_reuse)."""
+    """Sparse causal prefill attention over tile indices + diagonal (kascade_prefill_reuse;
+    the _f16 entry point when q, k, v are float16)."""
     B, Hq, N, d = q.shape
     Hkv = k.shape[1]
-    for name, t, dt in (("q", q, torch.bfloat16), ("k", k, torch.bfloat16), ("v", v, torch.bfloat16),
+    sfx = _data_suffix(q, k, v)
+    for name, t, dt in (("q", q, q.dtype), ("k", k, q.dtype), ("v", v, q.dtype),
                         ("idx", idx, torch.int32), ("idx_k", idx_k, torch.int32),
                         ("head_map", head_map, torch.int32)):
         _need_cuda(name, t, dt)
@@ -229,10 +247,10 @@ def prefill_reuse(q, k, v, idx, idx_k, head_map, scale: float, out=None, lse=Non
     shape = Shape(B, Hq, Hkv, d)
     need = _lib().kascade_prefill_reuse_workspace_bytes(shape, N, k_max)
     ws = workspace(need, dev) if ws is None else ws
-    rc = _lib().kascade_prefill_reuse(shape, int(N), _ptr(q), _ptr(k), _ptr(v), _ptr(idx),
+    rc = getattr(_lib(), "kascade_prefill_reuse" + sfx)(shape, int(N), _ptr(q), _ptr(k), _ptr(v), _ptr(idx),
                                       _ptr(idx_k), int(k_max), _ptr(head_map), float(scale),
                                       _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream())
-    check(rc, "kascade_prefill_reuse")
+    check(rc, "kascade_prefill_reuse" + sfx)
     return out, lse
 
 

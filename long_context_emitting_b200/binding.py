@@ -38,6 +38,10 @@ EXPORTS = (
     "kascade_prefill_anchor",
     "kascade_prefill_reuse_workspace_bytes",
     "kascade_prefill_reuse",
+    "kascade_decode_anchor_f16",
+    "kascade_decode_reuse_f16",
+    "kascade_prefill_anchor_f16",
+    "kascade_prefill_reuse_f16",
     "kascade_decode_anchor_paged",
     "kascade_decode_reuse_paged",
     "kascade_similarity_rows",
@@ -92,6 +96,10 @@ _SIGNATURES = {
     "kascade_get_device_status": (ctypes.c_int, [_P]),
     "kascade_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
+# fp16 variants take the same arguments as their bfloat16 counterparts
+for _name in ("kascade_decode_anchor", "kascade_decode_reuse", "kascade_prefill_anchor",
+              "kascade_prefill_reuse"):
+    _SIGNATURES[_name + "_f16"] = _SIGNATURES[_name]
 
 _lib = None
 

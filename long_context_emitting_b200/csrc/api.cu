@@ -86,11 +86,11 @@ size_t kascade_decode_anchor_workspace_bytes(kascade_shape s, int32_t max_T) {
   return decode_workspace_bytes(s.B, s.Hkv, s.Hq / s.Hkv, max_T, true);
 }
 
-int kascade_decode_anchor(kascade_shape s, const uint16_t* q, const uint16_t* k,
+static int kascade_decode_anchor_impl(kascade_shape s, const uint16_t* q, const uint16_t* k,
                           const uint16_t* v, const int64_t* kv_off, const int32_t* seq_len,
                           int32_t max_T, float scale, uint16_t* out, float* lse,
                           float* pooled, int64_t ld_pooled, void* ws, size_t ws_bytes,
-                          void* stream) {
+                          void* stream, bool f16) {
   int rc = check_shape(s);
   if (rc) return rc;
   if (max_T < 0 || ld_pooled < max_T || (ld_pooled & 3) || !std::isfinite(scale))
@@ -102,6 +102,7 @@ int kascade_decode_anchor(kascade_shape s, const uint16_t* q, const uint16_t* k,
     return KASCADE_ERR_INVALID_ARG;
   if (ws_bytes < kascade_decode_anchor_workspace_bytes(s, max_T)) return KASCADE_ERR_WORKSPACE_TOO_SMALL;
   DecodeParams p = {};
+  p.f16 = f16;
   p.B = s.B; p.Hq = s.Hq; p.Hkv = s.Hkv; p.G = s.Hq / s.Hkv;
   p.q = q; p.k = k; p.v = v; p.kv_off = kv_off; p.seq_len = seq_len; p.max_T = max_T;
   p.scale = scale; p.out = out; p.lse = lse; p.pooled = pooled; p.ld_pooled = ld_pooled;
@@ -111,16 +112,32 @@ int kascade_decode_anchor(kascade_shape s, const uint16_t* q, const uint16_t* k,
   return from_cuda(launch_decode_anchor(p, static_cast<cudaStream_t>(stream)));
 }
 
+int kascade_decode_anchor(kascade_shape s, const uint16_t* q, const uint16_t* k,
+                          const uint16_t* v, const int64_t* kv_off, const int32_t* seq_len,
+                          int32_t max_T, float scale, uint16_t* out, float* lse,
+                          float* pooled, int64_t ld_pooled, void* ws, size_t ws_bytes,
+                          void* stream) {
+  return kascade_decode_anchor_impl(s, q, k, v, kv_off, seq_len, max_T, scale, out, lse, pooled, ld_pooled, ws, ws_bytes, stream, false);
+}
+
+int kascade_decode_anchor_f16(kascade_shape s, const uint16_t* q, const uint16_t* k,
+                          const uint16_t* v, const int64_t* kv_off, const int32_t* seq_len,
+                          int32_t max_T, float scale, uint16_t* out, float* lse,
+                          float* pooled, int64_t ld_pooled, void* ws, size_t ws_bytes,
+                          void* stream) {
+  return kascade_decode_anchor_impl(s, q, k, v, kv_off, seq_len, max_T, scale, out, lse, pooled, ld_pooled, ws, ws_bytes, stream, true);
+}
+
 size_t kascade_decode_reuse_workspace_bytes(kascade_shape s, int32_t k_max) {
   if (check_shape(s) != KASCADE_OK || k_max < 0) return 0;
   return decode_workspace_bytes(s.B, s.Hkv, s.Hq / s.Hkv, k_max, false);
 }
 
-int kascade_decode_reuse(kascade_shape s, const uint16_t* q, const uint16_t* k,
+static int kascade_decode_reuse_impl(kascade_shape s, const uint16_t* q, const uint16_t* k,
                          const uint16_t* v, const int64_t* kv_off, const int32_t* seq_len,
                          const int32_t* idx, const int32_t* idx_k, int32_t k_max,
                          const int32_t* head_map, float scale, uint16_t* out, float* lse,
-                         void* ws, size_t ws_bytes, void* stream) {
+                         void* ws, size_t ws_bytes, void* stream, bool f16) {
   int rc = check_shape(s);
   if (rc) return rc;
   if (k_max < 0 || !std::isfinite(scale)) return KASCADE_ERR_INVALID_ARG;
@@ -134,6 +151,7 @@ int kascade_decode_reuse(kascade_shape s, const uint16_t* q, const uint16_t* k,
     return KASCADE_ERR_INVALID_ARG;
   if (ws_bytes < need) return KASCADE_ERR_WORKSPACE_TOO_SMALL;
   DecodeParams p = {};
+  p.f16 = f16;
   p.B = s.B; p.Hq = s.Hq; p.Hkv = s.Hkv; p.G = s.Hq / s.Hkv;
   p.q = q; p.k = k; p.v = v; p.kv_off = kv_off; p.seq_len = seq_len;
   p.max_T = 0x7fffffff;  // index validity is checked against each seq_len
@@ -142,6 +160,22 @@ int kascade_decode_reuse(kascade_shape s, const uint16_t* q, const uint16_t* k,
   p.status = device_status_ptr();
   if (!p.status) return KASCADE_ERR_CUDA;
   return from_cuda(launch_decode_reuse(p, static_cast<cudaStream_t>(stream)));
+}
+
+int kascade_decode_reuse(kascade_shape s, const uint16_t* q, const uint16_t* k,
+                         const uint16_t* v, const int64_t* kv_off, const int32_t* seq_len,
+                         const int32_t* idx, const int32_t* idx_k, int32_t k_max,
+                         const int32_t* head_map, float scale, uint16_t* out, float* lse,
+                         void* ws, size_t ws_bytes, void* stream) {
+  return kascade_decode_reuse_impl(s, q, k, v, kv_off, seq_len, idx, idx_k, k_max, head_map, scale, out, lse, ws, ws_bytes, stream, false);
+}
+
+int kascade_decode_reuse_f16(kascade_shape s, const uint16_t* q, const uint16_t* k,
+                         const uint16_t* v, const int64_t* kv_off, const int32_t* seq_len,
+                         const int32_t* idx, const int32_t* idx_k, int32_t k_max,
+                         const int32_t* head_map, float scale, uint16_t* out, float* lse,
+                         void* ws, size_t ws_bytes, void* stream) {
+  return kascade_decode_reuse_impl(s, q, k, v, kv_off, seq_len, idx, idx_k, k_max, head_map, scale, out, lse, ws, ws_bytes, stream, true);
 }
 
 // ------------------------------------------------------------ decode, paged --
@@ -286,9 +320,9 @@ size_t kascade_prefill_anchor_workspace_bytes(kascade_shape s, int32_t N) {
   return prefill_anchor_workspace_bytes(s.B, s.Hq, s.Hkv, N);
 }
 
-int kascade_prefill_anchor(kascade_shape s, int32_t N, const uint16_t* q, const uint16_t* k,
+static int kascade_prefill_anchor_impl(kascade_shape s, int32_t N, const uint16_t* q, const uint16_t* k,
                            const uint16_t* v, float scale, uint16_t* out, float* lse,
-                           float* pooled, void* ws, size_t ws_bytes, void* stream) {
+                           float* pooled, void* ws, size_t ws_bytes, void* stream, bool f16) {
   int rc = check_prefill(s, N);
   if (rc) return rc;
   if (!std::isfinite(scale) || !(scale > 0.f)) return KASCADE_ERR_INVALID_ARG;
@@ -300,6 +334,7 @@ int kascade_prefill_anchor(kascade_shape s, int32_t N, const uint16_t* q, const 
     return KASCADE_ERR_INVALID_ARG;
   if (ws_bytes < need) return KASCADE_ERR_WORKSPACE_TOO_SMALL;
   PrefillParams p = {};
+  p.f16 = f16;
   p.B = s.B; p.Hq = s.Hq; p.Hkv = s.Hkv; p.G = s.Hq / s.Hkv; p.N = N;
   p.q = q; p.k = k; p.v = v; p.scale = scale; p.out = out; p.lse = lse; p.pooled = pooled;
   p.ws = ws;
@@ -310,15 +345,27 @@ int kascade_prefill_anchor(kascade_shape s, int32_t N, const uint16_t* q, const 
   return from_cuda(e);
 }
 
+int kascade_prefill_anchor(kascade_shape s, int32_t N, const uint16_t* q, const uint16_t* k,
+                           const uint16_t* v, float scale, uint16_t* out, float* lse,
+                           float* pooled, void* ws, size_t ws_bytes, void* stream) {
+  return kascade_prefill_anchor_impl(s, N, q, k, v, scale, out, lse, pooled, ws, ws_bytes, stream, false);
+}
+
+int kascade_prefill_anchor_f16(kascade_shape s, int32_t N, const uint16_t* q, const uint16_t* k,
+                           const uint16_t* v, float scale, uint16_t* out, float* lse,
+                           float* pooled, void* ws, size_t ws_bytes, void* stream) {
+  return kascade_prefill_anchor_impl(s, N, q, k, v, scale, out, lse, pooled, ws, ws_bytes, stream, true);
+}
+
 size_t kascade_prefill_reuse_workspace_bytes(kascade_shape s, int32_t N, int32_t k_max) {
   if (check_prefill(s, N) != KASCADE_OK || k_max < 0) return 0;
   return prefill_reuse_workspace_bytes(s.B, s.Hq, s.Hkv, N, k_max);
 }
 
-int kascade_prefill_reuse(kascade_shape s, int32_t N, const uint16_t* q, const uint16_t* k,
+static int kascade_prefill_reuse_impl(kascade_shape s, int32_t N, const uint16_t* q, const uint16_t* k,
                           const uint16_t* v, const int32_t* idx, const int32_t* idx_k,
                           int32_t k_max, const int32_t* head_map, float scale, uint16_t* out,
-                          float* lse, void* ws, size_t ws_bytes, void* stream) {
+                          float* lse, void* ws, size_t ws_bytes, void* stream, bool f16) {
   int rc = check_prefill(s, N);
   if (rc) return rc;
   if (k_max < 0 || !std::isfinite(scale) || !(scale > 0.f)) return KASCADE_ERR_INVALID_ARG;
@@ -332,6 +379,7 @@ int kascade_prefill_reuse(kascade_shape s, int32_t N, const uint16_t* q, const u
     return KASCADE_ERR_INVALID_ARG;
   if (ws_bytes < need) return KASCADE_ERR_WORKSPACE_TOO_SMALL;
   PrefillParams p = {};
+  p.f16 = f16;
   p.B = s.B; p.Hq = s.Hq; p.Hkv = s.Hkv; p.G = s.Hq / s.Hkv; p.N = N;
   p.q = q; p.k = k; p.v = v; p.idx = idx; p.idx_k = idx_k; p.head_map = head_map;
   p.k_max = k_max; p.scale = scale; p.out = out; p.lse = lse; p.ws = ws;
@@ -340,6 +388,20 @@ int kascade_prefill_reuse(kascade_shape s, int32_t N, const uint16_t* q, const u
   cudaError_t e = launch_prefill_reuse(p, static_cast<cudaStream_t>(stream));
   if (e == cudaErrorNotSupported) return KASCADE_ERR_UNSUPPORTED_SHAPE;
   return from_cuda(e);
+}
+
+int kascade_prefill_reuse(kascade_shape s, int32_t N, const uint16_t* q, const uint16_t* k,
+                          const uint16_t* v, const int32_t* idx, const int32_t* idx_k,
+                          int32_t k_max, const int32_t* head_map, float scale, uint16_t* out,
+                          float* lse, void* ws, size_t ws_bytes, void* stream) {
+  return kascade_prefill_reuse_impl(s, N, q, k, v, idx, idx_k, k_max, head_map, scale, out, lse, ws, ws_bytes, stream, false);
+}
+
+int kascade_prefill_reuse_f16(kascade_shape s, int32_t N, const uint16_t* q, const uint16_t* k,
+                          const uint16_t* v, const int32_t* idx, const int32_t* idx_k,
+                          int32_t k_max, const int32_t* head_map, float scale, uint16_t* out,
+                          float* lse, void* ws, size_t ws_bytes, void* stream) {
+  return kascade_prefill_reuse_impl(s, N, q, k, v, idx, idx_k, k_max, head_map, scale, out, lse, ws, ws_bytes, stream, true);
 }
 
 }  // extern "C"

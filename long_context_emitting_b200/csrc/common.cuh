@@ -4,6 +4,7 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 namespace kascade {
 
@@ -71,6 +72,41 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ uint16_t to_bf16_bits(float x) {
   __nv_bfloat16 v = __float2bfloat16_rn(x);
   return *reinterpret_cast<uint16_t*>(&v);
+}
+
+// fp16 counterparts (the f16 entry points: same kernels, half-precision data)
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                              uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ uint16_t to_f16_bits(float x) {
+  __half v = __float2half_rn(x);
+  return *reinterpret_cast<uint16_t*>(&v);
+}
+// element-type dispatch: F16 = half precision, else bfloat16
+template <bool F16>
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+  if constexpr (F16) mma_f16_16816(d, a0, a1, a2, a3, b0, b1);
+  else mma_bf16_16816(d, a0, a1, a2, a3, b0, b1);
+}
+template <bool F16>
+__device__ __forceinline__ uint32_t pack_x2(float lo, float hi) {
+  if constexpr (F16) return pack_f16x2(lo, hi);
+  else return pack_bf16x2(lo, hi);
+}
+template <bool F16>
+__device__ __forceinline__ uint16_t to_bits(float x) {
+  if constexpr (F16) return to_f16_bits(x);
+  else return to_bf16_bits(x);
 }
 
 __device__ __forceinline__ float warp_max_xor_gid(float v) {

@@ -140,16 +140,16 @@ struct WarpState {
   float o[8][4];
 };
 
-template <bool GATHER>
+template <bool GATHER, bool F16>
 __device__ __forceinline__ void compute_blk(const Blk& x, WarpState& w, const uint32_t (&qf)[4][4],
                                             float scale_log2, float* lrow, int G, int tig) {
   // S^T = K · Q^T  (rows: items ia / ib; cols: heads 2tig, 2tig+1)
   float s[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};  // two independent chains
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    mma_bf16_16816(s, word_of(x.ka[j], 0), word_of(x.kb[j], 0), word_of(x.ka[j], 1),
+    mma_16816<F16>(s, word_of(x.ka[j], 0), word_of(x.kb[j], 0), word_of(x.ka[j], 1),
                    word_of(x.kb[j], 1), qf[j][0], qf[j][1]);
-    mma_bf16_16816(s2, word_of(x.ka[j], 2), word_of(x.kb[j], 2), word_of(x.ka[j], 3),
+    mma_16816<F16>(s2, word_of(x.ka[j], 2), word_of(x.kb[j], 2), word_of(x.ka[j], 3),
                    word_of(x.kb[j], 3), qf[j][2], qf[j][3]);
   }
 #pragma unroll
@@ -188,8 +188,8 @@ __device__ __forceinline__ void compute_blk(const Blk& x, WarpState& w, const ui
   }
 
   // O^T += V^T · P^T
-  const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p0, p1));
-  const uint32_t pb1 = movmatrix_trans(pack_bf16x2(p2, p3));
+  const uint32_t pb0 = movmatrix_trans(pack_x2<F16>(p0, p1));
+  const uint32_t pb1 = movmatrix_trans(pack_x2<F16>(p2, p3));
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
 #pragma unroll
@@ -198,7 +198,7 @@ __device__ __forceinline__ void compute_blk(const Blk& x, WarpState& w, const ui
       const uint32_t a1 = movmatrix_trans(word_of(x.va[j], 2 * pp + 1));
       const uint32_t a2 = movmatrix_trans(word_of(x.vb[j], 2 * pp));
       const uint32_t a3 = movmatrix_trans(word_of(x.vb[j], 2 * pp + 1));
-      mma_bf16_16816(w.o[2 * j + pp], a0, a1, a2, a3, pb0, pb1);
+      mma_16816<F16>(w.o[2 * j + pp], a0, a1, a2, a3, pb0, pb1);
     }
   }
 }
@@ -207,7 +207,7 @@ __device__ __forceinline__ void compute_blk(const Blk& x, WarpState& w, const ui
 // loads in flight during the current block's math), 2 CTAs per SM.  PAGED: a
 // warp's 16-token blocks start at multiples of 16 and the page size is a
 // multiple of 16, so each block lies in one page, looked up once per block.
-template <bool PAGED>
+template <bool PAGED, bool F16>
 __global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const SplitArgs a) {
   __shared__ float sm_o[kWarps][8][kHeadDim];
   __shared__ float sm_m[kWarps][8];
@@ -274,10 +274,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const SplitAr
   for (int i0 = i_begin; i0 < i_end; i0 += 32) {
     const bool has1 = i0 + 16 < i_end;
     if (has1) load(x1, i0 + 16);
-    compute_blk<false>(x0, ws, qf, a.scale_log2, lrow, G, tig);
+    compute_blk<false, F16>(x0, ws, qf, a.scale_log2, lrow, G, tig);
     if (!has1) break;
     if (i0 + 32 < i_end) load(x0, i0 + 32);
-    compute_blk<false>(x1, ws, qf, a.scale_log2, lrow, G, tig);
+    compute_blk<false, F16>(x1, ws, qf, a.scale_log2, lrow, G, tig);
   }
 
   // ---- merge the 4 warps of the CTA --------------------------------------
@@ -346,7 +346,7 @@ __device__ __forceinline__ uint32_t gswz(int r, int c) {
   return (uint32_t)r * 256u + ((uint32_t)(c ^ ((r & 1) << 2)) << 4);
 }
 
-template <bool PAGED>
+template <bool PAGED, bool F16>
 __global__ void __launch_bounds__(kThreads, 3) decode_gather_kernel(const SplitArgs a) {
   extern __shared__ uint8_t gsm_raw[];
   uint8_t* gsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gsm_raw) + 127) & ~uintptr_t(127));
@@ -459,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_gather_kernel(const SplitA
     x.okb = (m >> (gid + 8)) & 1u;
     x.ia = x.ib = 0;
     __syncwarp();                       // stage fully read before it is refilled
-    compute_blk<true>(x, ws, qf, a.scale_log2, nullptr, G, tig);
+    compute_blk<true, F16>(x, ws, qf, a.scale_log2, nullptr, G, tig);
   }
   cp_async_wait<0>();
 
@@ -527,7 +527,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_gather_kernel(const SplitA
           acc += f * *cluster.map_shared_rank(&sm_po[g][d], r);
         }
       }
-      a.out[((int64_t)b * a.Hq + h * G + g) * kHeadDim + d] = to_bf16_bits(L > 0.f ? acc / L : 0.f);
+      a.out[((int64_t)b * a.Hq + h * G + g) * kHeadDim + d] = to_bits<F16>(L > 0.f ? acc / L : 0.f);
       if (a.lse && d == 0) a.lse[(int64_t)b * a.Hq + h * G + g] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
     }
   }
@@ -547,6 +547,7 @@ struct CombineArgs {
   float* lse;
 };
 
+template <bool F16>
 __global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(const CombineArgs a) {
   __shared__ float s_M[8], s_L[8], s_lse2[8];
   const int b = blockIdx.z, h = blockIdx.y, chunk = blockIdx.x;
@@ -586,7 +587,7 @@ __global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(const C
           acc += fast_exp2(ml[(s * G + g) * 2] - M) * po[((int64_t)s * G + g) * kHeadDim + d];
         acc /= L;
       }
-      a.out[((int64_t)b * a.Hq + h * G + g) * kHeadDim + d] = to_bf16_bits(acc);
+      a.out[((int64_t)b * a.Hq + h * G + g) * kHeadDim + d] = to_bits<F16>(acc);
     }
     if (a.lse && threadIdx.x < G) {
       const float l2 = s_lse2[threadIdx.x];
@@ -725,7 +726,8 @@ static cudaError_t launch_decode(const DecodeParams& p, bool gather, cudaStream_
   dim3 grid(sp.nsplit, p.Hkv, p.B);
   if (gather) {
     // reuse: the nsplit CTAs of each (b, h) are one cluster and merge on chip
-    auto kern = paged ? decode_gather_kernel<true> : decode_gather_kernel<false>;
+    auto kern = paged ? (p.f16 ? decode_gather_kernel<true, true> : decode_gather_kernel<true, false>)
+                      : (p.f16 ? decode_gather_kernel<false, true> : decode_gather_kernel<false, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGSmem);
     if (e != cudaSuccess) return e;
     if (sp.nsplit > 8) {
@@ -748,8 +750,9 @@ static cudaError_t launch_decode(const DecodeParams& p, bool gather, cudaStream_
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }
-  if (paged) decode_split_kernel<true><<<grid, kThreads, 0, st>>>(a);
-  else decode_split_kernel<false><<<grid, kThreads, 0, st>>>(a);
+  auto split = paged ? (p.f16 ? decode_split_kernel<true, true> : decode_split_kernel<true, false>)
+                     : (p.f16 ? decode_split_kernel<false, true> : decode_split_kernel<false, false>);
+  split<<<grid, kThreads, 0, st>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
@@ -762,7 +765,8 @@ static cudaError_t launch_decode(const DecodeParams& p, bool gather, cudaStream_
   c.out = p.out; c.lse = p.lse;
   const int nchunk = max(1, (p.max_T + kPoolChunk - 1) / kPoolChunk);
   dim3 cgrid(nchunk, p.Hkv, p.B);
-  decode_combine_kernel<<<cgrid, kCombineThreads, 0, st>>>(c);
+  if (p.f16) decode_combine_kernel<true><<<cgrid, kCombineThreads, 0, st>>>(c);
+  else decode_combine_kernel<false><<<cgrid, kCombineThreads, 0, st>>>(c);
   return cudaGetLastError();
 }
 

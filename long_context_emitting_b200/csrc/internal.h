@@ -19,6 +19,7 @@ struct DecodeParams {
   const int64_t* kv_off;        // contiguous cache (NULL when paged)
   const int32_t* block_table;   // paged cache [B, max_pages] (NULL when contiguous)
   int max_pages = 0, page_size = 0, num_pages = 0;
+  bool f16 = false;             // q, k, v, out are fp16 (else bf16)
   const int32_t* seq_len;
   int max_T;
   // gather (reuse) only
@@ -55,6 +56,7 @@ cudaError_t launch_topk(const float* scores, int rows, int64_t ld, const int32_t
 // --------------------------------------------------------------- prefill ----
 struct PrefillParams {
   int B, Hq, Hkv, G, N;
+  bool f16 = false;  // q, k, v, out are fp16 (else bf16)
   const uint16_t* q;
   const uint16_t* k;
   const uint16_t* v;

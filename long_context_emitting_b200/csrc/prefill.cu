@@ -6,7 +6,7 @@
 // post-softmax pooling in prefill), 実装のポイント (128-query tiles),
 // 技術的詳細 › アンカーレイヤーと再利用レイヤー and › ヘッドリマッピング.
 //
-// prefill_attn_kernel<GATHER>
+// prefill_attn_kernel<GATHER, F16>  (F16: fp16 data, else bf16)
 //   One CTA per (query tile t, pair of query heads of one GQA group, sequence).
 //   The two heads share every K/V block, so each block is loaded once for two
 //   128 x 128 attention tiles.  Warp roles (384 threads, three warpgroups):
@@ -154,7 +154,7 @@ __device__ __forceinline__ constexpr uint64_t qpair_step(int ks) {
   return (uint64_t)(((uint32_t)(ks >> 2) * 4u * kHalfBytes + (uint32_t)(ks & 3) * 32u) >> 4);
 }
 
-template <bool GATHER>
+template <bool GATHER, bool F16>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
@@ -317,8 +317,8 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     } else if (warp == kMmaWarp) {
       // ================================ MMA issuer ==================================
       if (lane == 0) {
-        const uint32_t idesc_s = idesc_bf16(128, 128, false, false);
-        const uint32_t idesc_o = idesc_bf16(128, 128, false, true);
+        const uint32_t idesc_s = idesc_f16kind(128, 128, false, false, F16);
+        const uint32_t idesc_o = idesc_f16kind(128, 128, false, true, F16);
         // base descriptors: query tiles, and K / V of the two stages
         const uint64_t dq0 = kmajor_desc(sbase + kAttnQ, 0);
         const uint64_t dq1 = kmajor_desc(sbase + kAttnQ + kTileBytes, 0);
@@ -477,7 +477,7 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                       x0, x1);
             const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
             L[e2 & 3] = f2_add(L[e2 & 3], f2_pack(p0, p1));
-            pw[e2] = pack_bf16x2(p0, p1);
+            pw[e2] = pack_x2<F16>(p0, p1);
           }
           if (c == 2) {
             // keys 0..63 are stored: hand them to the MMA before the rest
@@ -513,10 +513,10 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
           for (int q8 = 0; q8 < 4; ++q8) {
             uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(o[8 * q8 + 0]) * inv_l, __uint_as_float(o[8 * q8 + 1]) * inv_l);
-            w.y = pack_bf16x2(__uint_as_float(o[8 * q8 + 2]) * inv_l, __uint_as_float(o[8 * q8 + 3]) * inv_l);
-            w.z = pack_bf16x2(__uint_as_float(o[8 * q8 + 4]) * inv_l, __uint_as_float(o[8 * q8 + 5]) * inv_l);
-            w.w = pack_bf16x2(__uint_as_float(o[8 * q8 + 6]) * inv_l, __uint_as_float(o[8 * q8 + 7]) * inv_l);
+            w.x = pack_x2<F16>(__uint_as_float(o[8 * q8 + 0]) * inv_l, __uint_as_float(o[8 * q8 + 1]) * inv_l);
+            w.y = pack_x2<F16>(__uint_as_float(o[8 * q8 + 2]) * inv_l, __uint_as_float(o[8 * q8 + 3]) * inv_l);
+            w.z = pack_x2<F16>(__uint_as_float(o[8 * q8 + 4]) * inv_l, __uint_as_float(o[8 * q8 + 5]) * inv_l);
+            w.w = pack_x2<F16>(__uint_as_float(o[8 * q8 + 6]) * inv_l, __uint_as_float(o[8 * q8 + 7]) * inv_l);
             *reinterpret_cast<uint4*>(orow + 32 * c + 8 * q8) = w;
           }
         }
@@ -532,6 +532,7 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   }
 }
 
+template <bool F16>
 __global__ void __launch_bounds__(kPoolThreads, 1)
 prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const PoolArgs a) {
@@ -636,7 +637,10 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // heads' summing warps have read the pair's previous tile.
         if (lane == 0) {
           const int np = hg >= 2 ? hg / 2 : 1;
-          const uint32_t idesc = idesc_bf16(128, hg >= 2 ? 256 : 128, false, false);
+          // Q and K in the data's type; the extra -lse step below is a separate
+          // instruction with bf16 operands on both sides
+          const uint32_t idesc = idesc_f16kind(128, hg >= 2 ? 256 : 128, false, false, F16);
+          const uint32_t idesc_x = idesc_bf16(128, hg >= 2 ? 256 : 128, false, false);
           bool ok = mbar_wait(bar(kPBarQ), rd & 1, a.status);
           for (int jb = 0; ok && jb < nblk; ++jb) {
             const int it = it0 + jb, st = it & 1;
@@ -650,7 +654,7 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
               for (int k16 = 0; k16 < 8; ++k16)
                 umma_ss(tmem + 256 * pr, dk + kmajor_step(k16), dq + qpair_step(k16), idesc, k16 > 0 ? 1u : 0u);
               umma_ss(tmem + 256 * pr, sw32_desc(sbase + kPoolKx), sw32_desc(sbase + kPoolQx + 2 * pr * kXBytes),
-                      idesc, 1u);
+                      idesc_x, 1u);
               umma_commit(bar(kPBarS + pr));
             }
             if (!ok) break;
@@ -788,14 +792,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // 2-D view [rows, 128] bf16, boxes of 64 columns x box_rows rows, 128-byte swizzle.
-bool make_tile_map(CUtensorMap* map, const void* base, uint64_t rows, uint32_t box_rows) {
+bool make_tile_map(CUtensorMap* map, const void* base, uint64_t rows, uint32_t box_rows, bool f16) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * 2};
   cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+  CUresult r = fn(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -811,8 +815,8 @@ static cudaError_t launch_attn(const PrefillParams& p, bool gather, cudaStream_t
   const uint64_t kv_rows = (uint64_t)p.B * p.Hkv * p.N;
   if (kv_rows >= (1ull << 31) || (uint64_t)p.B * p.Hq * p.N >= (1ull << 31)) return cudaErrorNotSupported;
   CUtensorMap tq, tk, tv;
-  if (!make_tile_map(&tq, p.q, (uint64_t)p.B * p.Hq * p.N, 128) || !make_tile_map(&tk, p.k, kv_rows, 128) ||
-      !make_tile_map(&tv, p.v, kv_rows, 128))
+  if (!make_tile_map(&tq, p.q, (uint64_t)p.B * p.Hq * p.N, 128, p.f16) ||
+      !make_tile_map(&tk, p.k, kv_rows, 128, p.f16) || !make_tile_map(&tv, p.v, kv_rows, 128, p.f16))
     return cudaErrorInvalidValue;
   AttnArgs a;
   a.B = p.B; a.Hq = p.Hq; a.Hkv = p.Hkv; a.G = p.G; a.N = p.N; a.n_tiles = n_tiles;
@@ -825,20 +829,15 @@ static cudaError_t launch_attn(const PrefillParams& p, bool gather, cudaStream_t
   // The kernel's setmaxnreg split assumes exactly kLaunchRegs registers per
   // thread at launch; with fewer, the softmax warpgroups' increase could never
   // be satisfied.  Refuse to launch a build that does not match.
+  auto kern = gather ? (p.f16 ? prefill_attn_kernel<true, true> : prefill_attn_kernel<true, false>)
+                     : (p.f16 ? prefill_attn_kernel<false, true> : prefill_attn_kernel<false, false>);
   cudaFuncAttributes fa;
-  cudaError_t e = gather ? cudaFuncGetAttributes(&fa, prefill_attn_kernel<true>)
-                         : cudaFuncGetAttributes(&fa, prefill_attn_kernel<false>);
+  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
   if (e != cudaSuccess) return e;
   if (fa.numRegs != kLaunchRegs) return cudaErrorNotSupported;
-  if (gather) {
-    e = cudaFuncSetAttribute(prefill_attn_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem);
-    if (e != cudaSuccess) return e;
-    prefill_attn_kernel<true><<<grid, kAttnThreads, kAttnSmem, st>>>(tq, tk, tv, a);
-  } else {
-    e = cudaFuncSetAttribute(prefill_attn_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem);
-    if (e != cudaSuccess) return e;
-    prefill_attn_kernel<false><<<grid, kAttnThreads, kAttnSmem, st>>>(tq, tk, tv, a);
-  }
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kAttnThreads, kAttnSmem, st>>>(tq, tk, tv, a);
   return cudaGetLastError();
 }
 
@@ -848,22 +847,23 @@ cudaError_t launch_prefill_anchor(const PrefillParams& p, cudaStream_t st) {
   const int n_tiles = p.N / kTile;
   if (n_tiles < 2) return cudaSuccess;
   CUtensorMap tq, tk;
-  if (!make_tile_map(&tq, p.q, (uint64_t)p.B * p.Hq * p.N, 128) ||
-      !make_tile_map(&tk, p.k, (uint64_t)p.B * p.Hkv * p.N, 128))
+  if (!make_tile_map(&tq, p.q, (uint64_t)p.B * p.Hq * p.N, 128, p.f16) ||
+      !make_tile_map(&tk, p.k, (uint64_t)p.B * p.Hkv * p.N, 128, p.f16))
     return cudaErrorInvalidValue;
   PoolArgs a;
   a.B = p.B; a.Hq = p.Hq; a.Hkv = p.Hkv; a.G = p.G; a.N = p.N; a.n_tiles = n_tiles;
   a.scale_log2 = (float)((double)p.scale * 1.4426950408889634);
   a.inv_scale = (float)(1.0 / (double)p.scale);
   a.lse = p.lse; a.pooled = p.pooled; a.status = p.status;
+  auto pool = p.f16 ? prefill_pool_kernel<true> : prefill_pool_kernel<false>;
   cudaFuncAttributes fa;  // the setmaxnreg split assumes kPoolLaunchRegs at launch
-  e = cudaFuncGetAttributes(&fa, prefill_pool_kernel);
+  e = cudaFuncGetAttributes(&fa, pool);
   if (e != cudaSuccess) return e;
   if (fa.numRegs != kPoolLaunchRegs) return cudaErrorNotSupported;
-  e = cudaFuncSetAttribute(prefill_pool_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPoolSmem);
+  e = cudaFuncSetAttribute(pool, cudaFuncAttributeMaxDynamicSharedMemorySize, kPoolSmem);
   if (e != cudaSuccess) return e;
   dim3 grid(n_tiles - 1, p.Hkv, p.B);
-  prefill_pool_kernel<<<grid, kPoolThreads, kPoolSmem, st>>>(tq, tk, a);
+  pool<<<grid, kPoolThreads, kPoolSmem, st>>>(tq, tk, a);
   return cudaGetLastError();
 }
 

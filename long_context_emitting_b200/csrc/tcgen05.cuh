@@ -288,13 +288,19 @@ __host__ __device__ constexpr uint32_t sw32_chunk_offset(int r, int c) {
 }
 
 // Instruction descriptor: kind::f16, bf16 x bf16 -> fp32, M x N, operand majors.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
-  return (1u << 4)                       // D format: f32
-         | (1u << 7)                     // A format: bf16
-         | (1u << 10)                    // B format: bf16
+// f16 = true: A and B are fp16 (format 0) instead of bf16 (format 1); both
+// operands of one instruction always share a type.
+__host__ __device__ constexpr uint32_t idesc_f16kind(int M, int N, bool a_mn_major, bool b_mn_major,
+                                                     bool f16) {
+  return (1u << 4)                              // D format: f32
+         | ((f16 ? 0u : 1u) << 7)               // A format
+         | ((f16 ? 0u : 1u) << 10)              // B format
          | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16)
-         | ((uint32_t)(N >> 3) << 17)    // N / 8
-         | ((uint32_t)(M >> 4) << 24);   // M / 16
+         | ((uint32_t)(N >> 3) << 17)           // N / 8
+         | ((uint32_t)(M >> 4) << 24);          // M / 16
+}
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return idesc_f16kind(M, N, a_mn_major, b_mn_major, false);
 }
 
 }  // namespace kascade

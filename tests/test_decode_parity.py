@@ -27,18 +27,25 @@ def _host_caches(cfg, inp, seqs):
     return [_np(ks[b]) for b in seqs], [_np(vs[b]) for b in seqs]
 
 
-def _check_layer_pair(cfg, seqs=None, reuse_layer=1):
-    """One anchor layer (0) and one reuse layer through the schedule, checked on `seqs`."""
+def _as(inp, dtype):
+    for name in ("q", "k", "v"):
+        inp[name] = inp[name].to(dtype)
+    return inp
+
+
+def _check_layer_pair(cfg, seqs=None, reuse_layer=1, dtype=torch.bfloat16):
+    """One anchor layer (0) and one reuse layer through the schedule, checked on `seqs`
+    (inputs and outputs in `dtype`: the bfloat16 or the float16 entry points)."""
     lens = cfg.seq_lens()
     seqs = list(range(cfg.B)) if seqs is None else seqs
     sch = DecodeSchedule(cfg.B, cfg.Hq, cfg.Hkv, lens, anchors=(0,), n_layers=2, device=DEV)
-    a_in = workload.decode_layer(cfg, 0, DEV)
-    out_a = torch.empty(cfg.B, cfg.Hq, cfg.d, dtype=torch.bfloat16, device=DEV)
+    a_in = _as(workload.decode_layer(cfg, 0, DEV), dtype)
+    out_a = torch.empty(cfg.B, cfg.Hq, cfg.d, dtype=dtype, device=DEV)
     sch.run_anchor(a_in, out_a)
     lse_a = sch.lse.clone()
     sch.run_topk()
     hm = workload.head_map(cfg, reuse_layer).to(DEV)
-    r_in = workload.decode_layer(cfg, reuse_layer, DEV)
+    r_in = _as(workload.decode_layer(cfg, reuse_layer, DEV), dtype)
     out_r = torch.empty_like(out_a)
     sch.run_reuse(r_in, hm, out_r)
     assert api.device_status() == 0
@@ -85,6 +92,12 @@ def test_decode_small_ragged():
     cfg = workload.scaled(workload.DECODE_4K, name="decode_small_ragged", B=8, T=None,
                           T_list=(1, 15, 16, 17, 127, 129, 1000, 2051))
     _check_layer_pair(cfg)
+
+
+def test_decode_small_ragged_f16():
+    cfg = workload.scaled(workload.DECODE_4K, name="decode_small_ragged", B=8, T=None,
+                          T_list=(1, 15, 16, 17, 127, 129, 1000, 2051))
+    _check_layer_pair(cfg, dtype=torch.float16)
 
 
 def test_decode_b1_t262144():

@@ -25,18 +25,22 @@ def _rows(tiles):
     return np.concatenate([np.arange(TILE * t, TILE * t + TILE) for t in tiles])
 
 
-def _check(cfg, tiles=None, reuse_layer=1, b=0):
+def _as(inp, dtype):
+    return {n: t.to(dtype) for n, t in inp.items()}
+
+
+def _check(cfg, tiles=None, reuse_layer=1, b=0, dtype=torch.bfloat16):
     N = cfg.N
     nt = N // TILE
     tiles = list(range(nt)) if tiles is None else tiles
     sch = PrefillSchedule(cfg.B, cfg.Hq, cfg.Hkv, N, (0,), 2, DEV)
-    a_in = workload.prefill_layer(cfg, 0, DEV)
+    a_in = _as(workload.prefill_layer(cfg, 0, DEV), dtype)
     out_a = torch.empty_like(a_in["q"])
     sch.run_anchor(a_in, out_a)
     lse_a = sch.lse.clone()
     sch.run_topk()
     hm = workload.head_map(cfg, reuse_layer).to(DEV)
-    r_in = workload.prefill_layer(cfg, reuse_layer, DEV)
+    r_in = _as(workload.prefill_layer(cfg, reuse_layer, DEV), dtype)
     out_r = torch.empty_like(r_in["q"])
     sch.run_reuse(r_in, hm, out_r)
     assert api.device_status() == 0
@@ -86,6 +90,13 @@ def test_prefill_gqa_group_sizes(Hq, Hkv):
     # pair of heads), G = 8 (two pooling rounds of four heads)
     cfg = workload.scaled(workload.PREFILL_16K, name=f"prefill_g{Hq // Hkv}", N=512, Hq=Hq, Hkv=Hkv)
     _check(cfg)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(32, 8), (8, 8), (16, 8), (32, 4)])
+def test_prefill_f16(Hq, Hkv):
+    # the float16 entry points (the evaluation's precision), whole small inputs
+    cfg = workload.scaled(workload.PREFILL_16K, name=f"prefill_f16_g{Hq // Hkv}", N=640, Hq=Hq, Hkv=Hkv)
+    _check(cfg, dtype=torch.float16)
 
 
 def test_prefill_batch2():
