@@ -669,9 +669,9 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   } else {
     setmaxnreg_inc<kPoolSumRegs>();
     // ------------------- summing warpgroups (one head each) -------------------
-    // Thread = key (TMEM lane).  The head's 128 scores are read in two halves
-    // of 64 queries; the tile is released to the MMA once the second half is in
-    // registers, before its exponentials are summed.
+    // Thread = key (TMEM lane).  The head's 128 scores are read 16 queries at
+    // a time, one load ahead of the summing; the tile is released to the MMA
+    // once the last columns are in registers, before they are summed.
     const int g = (warp >> 2) - 1;  // head of the round handled by this warpgroup
     const int key = (warp & 3) * 32 + lane;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
@@ -701,25 +701,21 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       for (int jb = 0; jb < nblk; ++jb) {
         const int it = it0 + jb;
         uint64_t A[4] = {0ull, 0ull, 0ull, 0ull};
-        // sum over 64 queries of exp2(sc * (q.k - lse/scale)), two per packed
+        // sum over 16 queries of exp2(sc * (q.k - lse/scale)), two per packed
         // instruction; 2 of every 8 pairs on the FMA pipe, the rest on the SFU
-        auto sum_half = [&](const uint32_t (&v)[2][32]) {
+        auto sum16 = [&](const uint32_t (&v)[16]) {
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-#pragma unroll
-            for (int e2 = 0; e2 < 16; ++e2) {
-              float x0, x1;
-              f2_unpack(f2_mul(f2_pack(__uint_as_float(v[c][2 * e2]), __uint_as_float(v[c][2 * e2 + 1])), SC),
-                        x0, x1);
-              float p0, p1;
-              if ((e2 & 7) >= 6) {
-                exp2_poly5_x2(x0, x1, p0, p1);
-              } else {
-                p0 = fast_exp2(x0);
-                p1 = fast_exp2(x1);
-              }
-              A[e2 & 3] = f2_add(A[e2 & 3], f2_pack(p0, p1));
+          for (int e2 = 0; e2 < 8; ++e2) {
+            float x0, x1;
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(v[2 * e2]), __uint_as_float(v[2 * e2 + 1])), SC), x0, x1);
+            float p0, p1;
+            if (e2 >= 6) {
+              exp2_poly5_x2(x0, x1, p0, p1);
+            } else {
+              p0 = fast_exp2(x0);
+              p1 = fast_exp2(x1);
             }
+            A[e2 & 3] = f2_add(A[e2 & 3], f2_pack(p0, p1));
           }
         };
         if (g < hg) {
@@ -728,23 +724,32 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             break;
           }
           tc_fence_after();
+          // The head's 128 scores in eight loads of 16 columns: each load is in
+          // flight while the previous columns are summed (a wait covers every
+          // earlier load; the fence keeps the compiler from reading a register
+          // before it).  The tile goes back to the MMA once the last load landed.
           const uint32_t tS = tmem + 128 * g + lane_base;
-          uint32_t v[2][32];
-          tmem_ld32(tS, v[0]);
-          tmem_ld32(tS + 32, v[1]);
+          uint32_t v0[16], v1[16];
+          tmem_ld16(tS, v0);
           tmem_wait_ld();
-          reg_fence32(v[0]);
-          reg_fence32(v[1]);
-          sum_half(v);
-          tmem_ld32(tS + 64, v[0]);
-          tmem_ld32(tS + 96, v[1]);
-          tmem_wait_ld();
-          reg_fence32(v[0]);
-          reg_fence32(v[1]);
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(kPBarFree + g / 2));  // the tile may be refilled
-          sum_half(v);
+          reg_fence16(v0);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint32_t (&cur)[16] = (c & 1) ? v1 : v0;
+            uint32_t (&nxt)[16] = (c & 1) ? v0 : v1;
+            if (c < 7) {
+              tmem_ld16(tS + 16 * (c + 1), nxt);
+            } else {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(bar(kPBarFree + g / 2));  // the tile may be refilled
+            }
+            sum16(cur);
+            if (c < 7) {
+              tmem_wait_ld();
+              reg_fence16(nxt);
+            }
+          }
         }
         float a0, a1, a2, a3;
         f2_unpack(f2_add(A[0], A[1]), a0, a1);
