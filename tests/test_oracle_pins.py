@@ -329,6 +329,34 @@ def test_dp_uses_weights_and_similarity():
     assert O.select_anchors_dp(S0, 2)[0] == 3.0
 
 
+def test_dp_single_anchor_value_is_total_weight():
+    # sim = 1 everywhere above the diagonal: one anchor at layer 0 covers every
+    # layer, and the value is the sum of the covered layers' weights w_l
+    L = 4
+    w = [1.0, 2.0, 4.0, 8.0]
+    S = O.weighted_similarity_matrix(np.triu(np.ones((L, L))), w)
+    assert O.select_anchors_dp(S, 1) == (15.0, [0])
+
+
+def test_dp_ties_keep_earliest_anchors():
+    # every anchor set scores 0: the smallest i among equal maxima gives 0..M-1
+    for L, M in ((6, 3), (5, 5), (4, 1)):
+        assert O.select_anchors_dp(np.zeros((L, L)), M) == (0.0, list(range(M)))
+
+
+def test_head_remap_direction_hand_example():
+    # k = 1.  Reuse head 0 = [0.5, 0.4, 0.1] puts its top key at 0.  Anchor
+    # head 0's top key is 1, which recovers 0.4 / 0.5 = 0.8 of that mass;
+    # anchor head 1's top key 2 recovers 0.2.  The other direction,
+    # sim(reuse, anchor), would rank them 0.01 / 0.98 and 0.45 / 0.5 and pick
+    # head 1.  Anchor head 2 duplicates head 0: the tie goes to the lower head.
+    a0 = [0.01, 0.98, 0.01]
+    a1 = [0.45, 0.05, 0.5]
+    p_anchor = np.array([[a0], [a1], [a0]])
+    p_reuse = np.array([[[0.5, 0.4, 0.1]], [a1], [[0.2, 0.3, 0.5]]])
+    assert O.head_remap(p_anchor, p_reuse, 1).tolist() == [0, 1, 1]
+
+
 def test_head_remap_recovers_permutation():
     rng = np.random.default_rng(3)
     Hkv, Q, n, k = 4, 3, 40, 6
