@@ -46,7 +46,8 @@ typedef enum {
   KASCADE_ERR_WORKSPACE_TOO_SMALL = 3,
   KASCADE_ERR_CUDA = 4,               /* a launch or CUDA runtime call failed */
   KASCADE_ERR_BAD_INDEX = 5,          /* device side: index / head map / length out of range */
-  KASCADE_ERR_NONFINITE = 6           /* device side: NaN in a Top-k score row */
+  KASCADE_ERR_NONFINITE = 6,          /* device side: NaN in a Top-k score row */
+  KASCADE_ERR_TIMEOUT = 7             /* device side: a bounded wait inside a kernel gave up */
 } kascade_status;
 
 /* Attention shape shared by all calls.  B = batch, Hq = query heads,
@@ -286,9 +287,23 @@ int kascade_select_anchors(const double* S, int32_t L, int32_t M, int32_t* ancho
 
 /* ------------------------------------------------------------------------- */
 /* Waits for `stream`, then returns and clears the sticky device status of the
- * current device: KASCADE_OK, or the first of KASCADE_ERR_BAD_INDEX /
- * KASCADE_ERR_NONFINITE that a kernel recorded (KASCADE_ERR_CUDA if the wait fails). */
+ * current device.  The result is KASCADE_OK or one recorded code, chosen in this
+ * order: KASCADE_ERR_TIMEOUT, then KASCADE_ERR_BAD_INDEX, then
+ * KASCADE_ERR_NONFINITE.  It is KASCADE_ERR_CUDA if the wait fails.
+ * KASCADE_ERR_TIMEOUT means that a prefill kernel's bounded wait gave up after
+ * about 2 s; that call's outputs are incomplete, and the context stays usable. */
 int kascade_get_device_status(void* stream);
+
+/* Diagnostic for the failure path above.  Launches one CTA on `stream`.  Its
+ * first thread waits on an mbarrier that nothing ever arrives at, through the
+ * same bounded wait the prefill kernels use:
+ *   spin == 0  suspending try_wait polls (the softmax and summing warps' wait)
+ *   spin != 0  non-suspending test_wait polls (the MMA thread's wait)
+ * The wait gives up after about 2 s and records the timeout bit, so the next
+ * kascade_get_device_status returns KASCADE_ERR_TIMEOUT.  Returns
+ * KASCADE_ERR_CUDA if the launch fails.  No memory is read or written apart from
+ * the status word. */
+int kascade_selftest_wait_timeout(int32_t spin, void* stream);
 
 /* Human-readable name of a status code (static string). */
 const char* kascade_status_string(int status);

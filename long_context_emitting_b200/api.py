@@ -65,6 +65,14 @@ def device_status(stream: Optional[int] = None) -> int:
     return int(_lib().kascade_get_device_status(_stream() if stream is None else stream))
 
 
+def selftest_wait_timeout(spin: bool = False, stream: Optional[int] = None) -> int:
+    """Run the bounded-wait diagnostic (about 2 s on the GPU) and return the
+    device status it leaves: KASCADE_ERR_TIMEOUT when the wait gave up."""
+    st = _stream() if stream is None else stream
+    check(_lib().kascade_selftest_wait_timeout(1 if spin else 0, st), "kascade_selftest_wait_timeout")
+    return device_status(st)
+
+
 def workspace(nbytes: int, device) -> torch.Tensor:
     return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device)
 

@@ -22,7 +22,9 @@ STATUS_NAMES = {
     4: "KASCADE_ERR_CUDA",
     5: "KASCADE_ERR_BAD_INDEX",
     6: "KASCADE_ERR_NONFINITE",
+    7: "KASCADE_ERR_TIMEOUT",
 }
+KASCADE_ERR_TIMEOUT = 7
 
 # Every symbol the header declares (checked by the CPU tests).
 EXPORTS = (
@@ -48,6 +50,7 @@ EXPORTS = (
     "kascade_select_anchors",
     "kascade_get_device_status",
     "kascade_status_string",
+    "kascade_selftest_wait_timeout",
 )
 
 
@@ -95,6 +98,7 @@ _SIGNATURES = {
     "kascade_select_anchors": (ctypes.c_int, [_P, _I32, _I32, _P, _P]),
     "kascade_get_device_status": (ctypes.c_int, [_P]),
     "kascade_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "kascade_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_int32, _P]),
 }
 # fp16 variants take the same arguments as their bfloat16 counterparts
 for _name in ("kascade_decode_anchor", "kascade_decode_reuse", "kascade_prefill_anchor",

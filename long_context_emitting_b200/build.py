@@ -14,7 +14,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libkascade.so")
-SOURCES = ["api.cu", "decode.cu", "topk.cu", "prefill.cu", "noalloc.cu", "calib.cu"]
+SOURCES = ["api.cu", "decode.cu", "topk.cu", "prefill.cu", "noalloc.cu", "calib.cu", "selftest.cu"]
 HEADERS = ["common.cuh", "internal.h", "tcgen05.cuh", "exp2_poly.cuh", "f32x2.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -65,6 +65,7 @@ const char* kascade_status_string(int status) {
     case KASCADE_ERR_CUDA: return "KASCADE_ERR_CUDA";
     case KASCADE_ERR_BAD_INDEX: return "KASCADE_ERR_BAD_INDEX";
     case KASCADE_ERR_NONFINITE: return "KASCADE_ERR_NONFINITE";
+    case KASCADE_ERR_TIMEOUT: return "KASCADE_ERR_TIMEOUT";
     default: return "KASCADE_ERR_UNKNOWN";
   }
 }
@@ -75,9 +76,16 @@ int kascade_get_device_status(void* stream) {
   if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v)) != cudaSuccess) return KASCADE_ERR_CUDA;
   const unsigned zero = 0u;
   if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero)) != cudaSuccess) return KASCADE_ERR_CUDA;
+  if (v & kStatusTimeout) return KASCADE_ERR_TIMEOUT;
   if (v & kStatusBadIndex) return KASCADE_ERR_BAD_INDEX;
   if (v & kStatusNonFinite) return KASCADE_ERR_NONFINITE;
   return KASCADE_OK;
+}
+
+int kascade_selftest_wait_timeout(int32_t spin, void* stream) {
+  unsigned* status = device_status_ptr();
+  if (!status) return KASCADE_ERR_CUDA;
+  return from_cuda(launch_wait_timeout(spin != 0, status, static_cast<cudaStream_t>(stream)));
 }
 
 // ------------------------------------------------------------------ decode --

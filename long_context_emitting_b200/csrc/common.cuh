@@ -13,6 +13,7 @@ constexpr int kHeadDim = 128;
 // Bits of the sticky device status word (see kascade_get_device_status).
 constexpr unsigned kStatusBadIndex = 1u;
 constexpr unsigned kStatusNonFinite = 2u;
+constexpr unsigned kStatusTimeout = 4u;  // a bounded wait gave up
 
 __device__ __forceinline__ void flag_status(unsigned* status, unsigned bit) {
   if (status) atomicOr(status, bit);

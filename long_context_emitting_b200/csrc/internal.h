@@ -92,6 +92,11 @@ struct SimArgs {
   unsigned* status;
 };
 cudaError_t launch_similarity_rows(const SimArgs& a, int n_out, cudaStream_t st);
+
+// One CTA whose first thread waits on an mbarrier nothing arrives at, through
+// the prefill kernels' bounded wait (spin: the non-suspending variant); the
+// wait gives up after about 2 s and ORs the timeout bit into *status.
+cudaError_t launch_wait_timeout(bool spin, unsigned* status, cudaStream_t st);
 void select_anchors_dp(const double* S, int L, int M, int32_t* anchors, double* best);
 
 }  // namespace kascade

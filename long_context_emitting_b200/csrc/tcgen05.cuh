@@ -11,8 +11,6 @@
 
 namespace kascade {
 
-constexpr unsigned kStatusTimeout = 4u;
-
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -8,7 +8,8 @@ The GPU test calls it through the C ABI twice in a row, on different inputs
 and sizes (the array keeps the first call's contents), and checks each result
 against the regular kascade_decode_anchor with caller-provided scratch, within
 the tolerances the other parity tests use.  This file is named to be collected
-last; it passes alone in a fresh process and after the rest of the suite."""
+after the parity tests; it passes alone in a fresh process and after the rest
+of the suite."""
 import numpy as np
 import pytest
 import torch
