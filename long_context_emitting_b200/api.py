@@ -47,10 +47,6 @@ def _data_suffix(*ts) -> str:
     return "_f16" if dt == torch.float16 else ""
 
 
-def _bits(t: torch.Tensor) -> torch.Tensor:
-    return t.view(torch.int16) if t.dtype == torch.bfloat16 else t
-
-
 def _stream() -> int:
     return torch.cuda.current_stream().cuda_stream
 
