@@ -2,7 +2,7 @@
 
 Reuse outputs are checked twice: against the oracle fed the GPU's own
 indices (isolates the attention arithmetic) and end to end against the
-oracle's own indices (index differences judged by the relative rule)."""
+oracle's own indices (index differences checked by the relative rule)."""
 import numpy as np
 import pytest
 import torch
