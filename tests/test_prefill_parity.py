@@ -84,6 +84,15 @@ def test_prefill_small_all_tiles():
     _check(cfg)
 
 
+@pytest.mark.parametrize("N", [128, 256])
+def test_prefill_one_and_two_tiles(N):
+    # N = 128: a single tile with an empty prefix (k = 0; the pooling launch is
+    # skipped, and reuse is the diagonal block alone).  N = 256: tile 1's
+    # prefix is shorter than the 128 floor, so k is the whole prefix.
+    cfg = workload.scaled(workload.PREFILL_16K, name=f"prefill_n{N}", N=N)
+    _check(cfg)
+
+
 @pytest.mark.parametrize("Hq,Hkv", [(8, 8), (16, 8), (32, 4)])
 def test_prefill_gqa_group_sizes(Hq, Hkv):
     # G = 1 (one tile per CTA; pooling with a single N = 128 head), G = 2 (one
