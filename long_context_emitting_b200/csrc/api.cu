@@ -7,6 +7,7 @@
 
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 
@@ -20,16 +21,20 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
+// Device address of the status word on the current device, looked up once per
+// device; threads that race on a first call all store the same address.
 unsigned* device_status_ptr() {
-  static unsigned* cache[kMaxDevices] = {};
+  static std::atomic<unsigned*> cache[kMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  if (!cache[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
-    cache[dev] = static_cast<unsigned*>(p);
+  unsigned* p = cache[dev].load(std::memory_order_acquire);
+  if (!p) {
+    void* q = nullptr;
+    if (cudaGetSymbolAddress(&q, g_device_status) != cudaSuccess) return nullptr;
+    p = static_cast<unsigned*>(q);
+    cache[dev].store(p, std::memory_order_release);
   }
-  return cache[dev];
+  return p;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }

@@ -10,6 +10,8 @@
 
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 namespace kascade {
 
 static __device__ __align__(256) unsigned char g_static_scratch[KASCADE_STATIC_SCRATCH_BYTES];
@@ -22,17 +24,18 @@ constexpr int kMaxDevices = 64;
 
 // Device address of g_static_scratch on the current device, looked up on the
 // first call per device (the lookup may load the module on that device, which
-// is why the first call should not happen inside a stream capture).
+// is why the first call should not happen inside a stream capture).  Threads
+// that race on a first call all store the same address.
 void* static_scratch_address() {
-  static void* cache[kMaxDevices] = {};
+  static std::atomic<void*> cache[kMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  if (!cache[dev]) {
-    void* p = nullptr;
+  void* p = cache[dev].load(std::memory_order_acquire);
+  if (!p) {
     if (cudaGetSymbolAddress(&p, kascade::g_static_scratch) != cudaSuccess) return nullptr;
-    cache[dev] = p;
+    cache[dev].store(p, std::memory_order_release);
   }
-  return cache[dev];
+  return p;
 }
 
 }  // namespace
