@@ -42,7 +42,8 @@ extern "C" {
 typedef enum {
   KASCADE_OK = 0,
   KASCADE_ERR_INVALID_ARG = 1,        /* NULL/misaligned pointer, negative size, k > length ... */
-  KASCADE_ERR_UNSUPPORTED_SHAPE = 2,  /* d != 128, group > 8, prefill N not a multiple of 128 */
+  KASCADE_ERR_UNSUPPORTED_SHAPE = 2,  /* d != 128, group > 8, prefill N not a multiple of 128,
+                                         decode anchor with B·Hq·max_T > 2^46 */
   KASCADE_ERR_WORKSPACE_TOO_SMALL = 3,
   KASCADE_ERR_CUDA = 4,               /* a launch or CUDA runtime call failed */
   KASCADE_ERR_BAD_INDEX = 5,          /* device side: index / head map / length out of range */
@@ -82,7 +83,9 @@ int32_t kascade_k_for_len(int32_t n);
  *   pooled  fp32 [B, Hkv, ld_pooled], ld_pooled >= max_T, ld_pooled % 4 == 0; entries at
  *           t >= T_b are left untouched
  *   ws      scratch of at least kascade_decode_anchor_workspace_bytes(s, max_T) bytes
- * A sequence with T_b == 0 gets out = 0 and lse = -inf. */
+ * A sequence with T_b == 0 gets out = 0 and lse = -inf.  Shapes with B·Hq·max_T > 2^46 are
+ * refused (KASCADE_ERR_UNSUPPORTED_SHAPE; the workspace query returns 0), so that no
+ * workspace size can wrap around. */
 size_t kascade_decode_anchor_workspace_bytes(kascade_shape s, int32_t max_T);
 int kascade_decode_anchor(kascade_shape s, const uint16_t* q, const uint16_t* k,
                           const uint16_t* v, const int64_t* kv_off, const int32_t* seq_len,

@@ -50,6 +50,14 @@ int check_shape(const kascade_shape& s) {
 
 int from_cuda(cudaError_t e) { return e == cudaSuccess ? KASCADE_OK : KASCADE_ERR_CUDA; }
 
+// The decode anchor's workspace holds B·Hq·max_T fp32 logits plus smaller
+// partials.  Shapes past 2^46 logits (256 TiB) are refused, so no workspace
+// size computation can wrap around.
+bool decode_logits_too_large(const kascade_shape& s, int32_t max_T) {
+  const uint64_t heads = (uint64_t)s.B * (uint64_t)s.Hq;  // < 2^62
+  return heads != 0 && (uint64_t)max_T > (1ull << 46) / heads;
+}
+
 }  // namespace
 
 extern "C" {
@@ -95,7 +103,7 @@ int kascade_selftest_wait_timeout(int32_t spin, void* stream) {
 
 // ------------------------------------------------------------------ decode --
 size_t kascade_decode_anchor_workspace_bytes(kascade_shape s, int32_t max_T) {
-  if (check_shape(s) != KASCADE_OK || max_T < 0) return 0;
+  if (check_shape(s) != KASCADE_OK || max_T < 0 || decode_logits_too_large(s, max_T)) return 0;
   return decode_workspace_bytes(s.B, s.Hkv, s.Hq / s.Hkv, max_T, true);
 }
 
@@ -108,6 +116,7 @@ static int kascade_decode_anchor_impl(kascade_shape s, const uint16_t* q, const 
   if (rc) return rc;
   if (max_T < 0 || ld_pooled < max_T || (ld_pooled & 3) || !std::isfinite(scale))
     return KASCADE_ERR_INVALID_ARG;
+  if (decode_logits_too_large(s, max_T)) return KASCADE_ERR_UNSUPPORTED_SHAPE;
   if (s.B == 0) return KASCADE_OK;
   if (!q || !k || !v || !kv_off || !seq_len || !out || !pooled || !ws) return KASCADE_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(pooled) ||
@@ -211,6 +220,7 @@ int kascade_decode_anchor_paged(kascade_shape s, const uint16_t* q, const uint16
   if (rc) return rc;
   if (max_T < 0 || ld_pooled < max_T || (ld_pooled & 3) || !std::isfinite(scale))
     return KASCADE_ERR_INVALID_ARG;
+  if (decode_logits_too_large(s, max_T)) return KASCADE_ERR_UNSUPPORTED_SHAPE;
   if (s.B == 0) return KASCADE_OK;
   if ((rc = check_pages(k_pages, v_pages, block_table, num_pages, max_pages, page_size))) return rc;
   if ((int64_t)max_pages * page_size < max_T) return KASCADE_ERR_INVALID_ARG;

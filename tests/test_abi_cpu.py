@@ -85,6 +85,20 @@ def test_prefill_scale_must_be_positive(lib):
         assert lib.kascade_prefill_reuse(s, 256, P, P, P, P, P, 8, P, bad, P, P, P, ws, None) == INVALID
 
 
+def test_oversized_decode_workspace_is_refused(lib):
+    # B·Hq·max_T past 2^46 logits: refused on the host, so no workspace size
+    # computation can wrap around to a small number
+    huge = Shape(65535, 32, 8, 128)
+    T = 2**31 - 1
+    assert lib.kascade_decode_anchor_workspace_bytes(huge, T) == 0
+    assert lib.kascade_decode_anchor(huge, P, P, P, P, P, T, 0.1, P, P, P, 2**31, P, 1 << 60,
+                                     None) == UNSUPPORTED
+    assert lib.kascade_decode_anchor_static_ws(huge, P, P, P, P, P, T, 0.1, P, P, P, 2**31,
+                                               None) == UNSUPPORTED
+    # the largest shapes in use stay accepted
+    assert lib.kascade_decode_anchor_workspace_bytes(Shape(64, 32, 8, 128), 131072) > 0
+
+
 def test_workspace_too_small(lib):
     s = Shape(4, 32, 8, 128)
     need = lib.kascade_decode_anchor_workspace_bytes(s, 32768)
