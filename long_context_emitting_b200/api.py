@@ -36,6 +36,22 @@ def _need_cuda(name: str, t: torch.Tensor, dtype: torch.dtype) -> None:
         raise ValueError(f"{name} must be contiguous")
 
 
+def _need_size(name: str, t: torch.Tensor, dtype: torch.dtype, n: int) -> None:
+    """A contiguous CUDA tensor of ``dtype`` with at least ``n`` elements: the
+    kernels read or write that many from its start, and nothing checks the
+    size below this layer."""
+    _need_cuda(name, t, dtype)
+    if t.numel() < n:
+        raise ValueError(f"{name} has {t.numel()} elements; this call needs at least {n}")
+
+
+def _ws_bytes(ws: torch.Tensor) -> int:
+    """Byte size of a caller's workspace tensor (any dtype)."""
+    if not isinstance(ws, torch.Tensor) or not ws.is_cuda or not ws.is_contiguous():
+        raise ValueError("ws must be a contiguous CUDA tensor")
+    return ws.numel() * ws.element_size()
+
+
 _DATA_DTYPES = (torch.bfloat16, torch.float16)
 
 
@@ -86,20 +102,23 @@ def decode_anchor(q, k, v, kv_off, seq_len, max_T: int, scale: float, Hkv: int,
     sfx = _data_suffix(q, k, v)
     for name, t in (("q", q), ("k", k), ("v", v)):
         _need_cuda(name, t, q.dtype)
-    _need_cuda("kv_off", kv_off, torch.int64)
-    _need_cuda("seq_len", seq_len, torch.int32)
+    _need_size("kv_off", kv_off, torch.int64, B)
+    _need_size("seq_len", seq_len, torch.int32, B)
     dev = q.device
     if ld_pooled is None:
         ld_pooled = (max_T + 3) // 4 * 4
     out = torch.empty(B, Hq, d, dtype=q.dtype, device=dev) if out is None else out
     lse = torch.empty(B, Hq, dtype=torch.float32, device=dev) if lse is None else lse
     pooled = torch.empty(B, Hkv, ld_pooled, dtype=torch.float32, device=dev) if pooled is None else pooled
+    _need_size("out", out, q.dtype, B * Hq * d)
+    _need_size("lse", lse, torch.float32, B * Hq)
+    _need_size("pooled", pooled, torch.float32, B * Hkv * ld_pooled)
     shape = Shape(B, Hq, Hkv, d)
     need = _lib().kascade_decode_anchor_workspace_bytes(shape, max_T)
     ws = workspace(need, dev) if ws is None else ws
     rc = getattr(_lib(), "kascade_decode_anchor" + sfx)(shape, _ptr(q), _ptr(k), _ptr(v), _ptr(kv_off), _ptr(seq_len),
                                       int(max_T), float(scale), _ptr(out), _ptr(lse), _ptr(pooled),
-                                      int(ld_pooled), _ptr(ws), ws.numel(), _stream())
+                                      int(ld_pooled), _ptr(ws), _ws_bytes(ws), _stream())
     check(rc, "kascade_decode_anchor" + sfx)
     return out, lse, pooled
 
@@ -114,50 +133,69 @@ def decode_reuse(q, k, v, kv_off, seq_len, idx, idx_k, head_map, scale: float, H
     the _f16 entry point when q, k, v are float16)."""
     B, Hq, d = q.shape
     sfx = _data_suffix(q, k, v)
-    for name, t, dt in (("q", q, q.dtype), ("k", k, q.dtype), ("v", v, q.dtype),
-                        ("kv_off", kv_off, torch.int64), ("seq_len", seq_len, torch.int32),
-                        ("idx", idx, torch.int32), ("idx_k", idx_k, torch.int32),
-                        ("head_map", head_map, torch.int32)):
-        _need_cuda(name, t, dt)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need_cuda(name, t, q.dtype)
     k_max = idx.shape[-1]
+    _need_size("kv_off", kv_off, torch.int64, B)
+    _need_size("seq_len", seq_len, torch.int32, B)
+    _need_size("idx", idx, torch.int32, B * Hkv * k_max)
+    _need_size("idx_k", idx_k, torch.int32, B * Hkv)
+    _need_size("head_map", head_map, torch.int32, Hkv)
     dev = q.device
     out = torch.empty(B, Hq, d, dtype=q.dtype, device=dev) if out is None else out
     lse = torch.empty(B, Hq, dtype=torch.float32, device=dev) if lse is None else lse
+    _need_size("out", out, q.dtype, B * Hq * d)
+    _need_size("lse", lse, torch.float32, B * Hq)
     shape = Shape(B, Hq, Hkv, d)
     need = _lib().kascade_decode_reuse_workspace_bytes(shape, k_max)
     ws = workspace(need, dev) if ws is None else ws
     rc = getattr(_lib(), "kascade_decode_reuse" + sfx)(shape, _ptr(q), _ptr(k), _ptr(v), _ptr(kv_off), _ptr(seq_len),
                                      _ptr(idx), _ptr(idx_k), int(k_max), _ptr(head_map),
-                                     float(scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                     float(scale), _ptr(out), _ptr(lse), _ptr(ws), _ws_bytes(ws),
                                      _stream())
     check(rc, "kascade_decode_reuse" + sfx)
     return out, lse
 
 
 # ------------------------------------------------------------ decode, paged ----
+def _need_pages(k_pages, v_pages, block_table, B: int, Hkv: int, page_size: int, d: int) -> None:
+    """Page store [num_pages, Hkv, page_size, d] (K and V alike) and a block
+    table with a row of page numbers for each of the B sequences."""
+    _need_cuda("k_pages", k_pages, torch.bfloat16)
+    _need_cuda("v_pages", v_pages, torch.bfloat16)
+    _need_cuda("block_table", block_table, torch.int32)
+    if k_pages.dim() != 4 or tuple(k_pages.shape[1:]) != (Hkv, page_size, d):
+        raise ValueError(f"k_pages must be [num_pages, {Hkv}, {page_size}, {d}], got {tuple(k_pages.shape)}")
+    if v_pages.shape != k_pages.shape:
+        raise ValueError("v_pages must have the shape of k_pages")
+    if block_table.dim() != 2 or block_table.shape[0] < B:
+        raise ValueError(f"block_table must be [>= {B}, max_pages], got {tuple(block_table.shape)}")
+
+
 def decode_anchor_paged(q, k_pages, v_pages, block_table, page_size: int, seq_len, max_T: int,
                         scale: float, Hkv: int, out=None, lse=None, pooled=None,
                         ld_pooled: Optional[int] = None, ws=None):
     """kascade_decode_anchor over a paged cache (see paging.to_paged)."""
     B, Hq, d = q.shape
     _need_cuda("q", q, torch.bfloat16)
-    _need_cuda("k_pages", k_pages, torch.bfloat16)
-    _need_cuda("v_pages", v_pages, torch.bfloat16)
-    _need_cuda("block_table", block_table, torch.int32)
-    _need_cuda("seq_len", seq_len, torch.int32)
+    _need_pages(k_pages, v_pages, block_table, B, Hkv, page_size, d)
+    _need_size("seq_len", seq_len, torch.int32, B)
     dev = q.device
     if ld_pooled is None:
         ld_pooled = (max_T + 3) // 4 * 4
     out = torch.empty(B, Hq, d, dtype=torch.bfloat16, device=dev) if out is None else out
     lse = torch.empty(B, Hq, dtype=torch.float32, device=dev) if lse is None else lse
     pooled = torch.empty(B, Hkv, ld_pooled, dtype=torch.float32, device=dev) if pooled is None else pooled
+    _need_size("out", out, torch.bfloat16, B * Hq * d)
+    _need_size("lse", lse, torch.float32, B * Hq)
+    _need_size("pooled", pooled, torch.float32, B * Hkv * ld_pooled)
     shape = Shape(B, Hq, Hkv, d)
     need = _lib().kascade_decode_anchor_workspace_bytes(shape, max_T)
     ws = workspace(need, dev) if ws is None else ws
     rc = _lib().kascade_decode_anchor_paged(
         shape, _ptr(q), _ptr(k_pages), _ptr(v_pages), int(k_pages.shape[0]), _ptr(block_table),
         int(block_table.shape[1]), int(page_size), _ptr(seq_len), int(max_T), float(scale),
-        _ptr(out), _ptr(lse), _ptr(pooled), int(ld_pooled), _ptr(ws), ws.numel(), _stream())
+        _ptr(out), _ptr(lse), _ptr(pooled), int(ld_pooled), _ptr(ws), _ws_bytes(ws), _stream())
     check(rc, "kascade_decode_anchor_paged")
     return out, lse, pooled
 
@@ -166,22 +204,25 @@ def decode_reuse_paged(q, k_pages, v_pages, block_table, page_size: int, seq_len
                        head_map, scale: float, Hkv: int, out=None, lse=None, ws=None):
     """kascade_decode_reuse over a paged cache (see paging.to_paged)."""
     B, Hq, d = q.shape
-    for name, t, dt in (("q", q, torch.bfloat16), ("k_pages", k_pages, torch.bfloat16),
-                        ("v_pages", v_pages, torch.bfloat16), ("block_table", block_table, torch.int32),
-                        ("seq_len", seq_len, torch.int32), ("idx", idx, torch.int32),
-                        ("idx_k", idx_k, torch.int32), ("head_map", head_map, torch.int32)):
-        _need_cuda(name, t, dt)
+    _need_cuda("q", q, torch.bfloat16)
+    _need_pages(k_pages, v_pages, block_table, B, Hkv, page_size, d)
     k_max = idx.shape[-1]
+    _need_size("seq_len", seq_len, torch.int32, B)
+    _need_size("idx", idx, torch.int32, B * Hkv * k_max)
+    _need_size("idx_k", idx_k, torch.int32, B * Hkv)
+    _need_size("head_map", head_map, torch.int32, Hkv)
     dev = q.device
     out = torch.empty(B, Hq, d, dtype=torch.bfloat16, device=dev) if out is None else out
     lse = torch.empty(B, Hq, dtype=torch.float32, device=dev) if lse is None else lse
+    _need_size("out", out, torch.bfloat16, B * Hq * d)
+    _need_size("lse", lse, torch.float32, B * Hq)
     shape = Shape(B, Hq, Hkv, d)
     need = _lib().kascade_decode_reuse_workspace_bytes(shape, k_max)
     ws = workspace(need, dev) if ws is None else ws
     rc = _lib().kascade_decode_reuse_paged(
         shape, _ptr(q), _ptr(k_pages), _ptr(v_pages), int(k_pages.shape[0]), _ptr(block_table),
         int(block_table.shape[1]), int(page_size), _ptr(seq_len), _ptr(idx), _ptr(idx_k),
-        int(k_max), _ptr(head_map), float(scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+        int(k_max), _ptr(head_map), float(scale), _ptr(out), _ptr(lse), _ptr(ws), _ws_bytes(ws),
         _stream())
     check(rc, "kascade_decode_reuse_paged")
     return out, lse
@@ -191,11 +232,12 @@ def decode_reuse_paged(q, k_pages, v_pages, block_table, page_size: int, seq_len
 def topk(scores, row_len, row_k, k_max: int, out=None):
     """Row-wise Top-k (ties to lower index, ascending output; tail = -1)."""
     _need_cuda("scores", scores, torch.float32)
-    _need_cuda("row_len", row_len, torch.int32)
-    _need_cuda("row_k", row_k, torch.int32)
     ld = scores.shape[-1]
     rows = scores.numel() // ld if ld else 0
+    _need_size("row_len", row_len, torch.int32, rows)
+    _need_size("row_k", row_k, torch.int32, rows)
     out = torch.empty(rows, k_max, dtype=torch.int32, device=scores.device) if out is None else out
+    _need_size("out", out, torch.int32, rows * k_max)
     rc = _lib().kascade_topk(_ptr(scores), int(rows), int(ld), _ptr(row_len), _ptr(row_k),
                              int(k_max), _ptr(out), None, 0, _stream())
     check(rc, "kascade_topk")
@@ -207,6 +249,14 @@ def prefill_anchor_workspace_bytes(B, Hq, Hkv, N) -> int:
     return int(_lib().kascade_prefill_anchor_workspace_bytes(Shape(B, Hq, Hkv, HEAD_DIM), N))
 
 
+def _need_kv_like(k, v, B: int, N: int, d: int) -> None:
+    """Prefill K and V as [B, Hkv, N, d], the same shape."""
+    if k.dim() != 4 or k.shape[0] != B or k.shape[2] != N or k.shape[3] != d:
+        raise ValueError(f"k must be [{B}, Hkv, {N}, {d}], got {tuple(k.shape)}")
+    if v.shape != k.shape:
+        raise ValueError("v must have the shape of k")
+
+
 def prefill_anchor(q, k, v, scale: float, out=None, lse=None, pooled=None, ws=None):
     """Dense causal prefill attention + tile-pooled probabilities (kascade_prefill_anchor;
     the _f16 entry point when q, k, v are float16)."""
@@ -215,16 +265,20 @@ def prefill_anchor(q, k, v, scale: float, out=None, lse=None, pooled=None, ws=No
     sfx = _data_suffix(q, k, v)
     for name, t in (("q", q), ("k", k), ("v", v)):
         _need_cuda(name, t, q.dtype)
+    _need_kv_like(k, v, B, N, d)
     dev = q.device
     out = torch.empty_like(q) if out is None else out
     lse = torch.empty(B, Hq, N, dtype=torch.float32, device=dev) if lse is None else lse
     if pooled is None:
         pooled = torch.empty(B, N // TILE, Hkv, N, dtype=torch.float32, device=dev)
+    _need_size("out", out, q.dtype, q.numel())
+    _need_size("lse", lse, torch.float32, B * Hq * N)
+    _need_size("pooled", pooled, torch.float32, B * (N // TILE) * Hkv * N)
     shape = Shape(B, Hq, Hkv, d)
     need = _lib().kascade_prefill_anchor_workspace_bytes(shape, N)
     ws = workspace(need, dev) if ws is None else ws
     rc = getattr(_lib(), "kascade_prefill_anchor" + sfx)(shape, int(N), _ptr(q), _ptr(k), _ptr(v), float(scale),
-                                       _ptr(out), _ptr(lse), _ptr(pooled), _ptr(ws), ws.numel(),
+                                       _ptr(out), _ptr(lse), _ptr(pooled), _ptr(ws), _ws_bytes(ws),
                                        _stream())
     check(rc, "kascade_prefill_anchor" + sfx)
     return out, lse, pooled
@@ -240,20 +294,25 @@ def prefill_reuse(q, k, v, idx, idx_k, head_map, scale: float, out=None, lse=Non
     B, Hq, N, d = q.shape
     Hkv = k.shape[1]
     sfx = _data_suffix(q, k, v)
-    for name, t, dt in (("q", q, q.dtype), ("k", k, q.dtype), ("v", v, q.dtype),
-                        ("idx", idx, torch.int32), ("idx_k", idx_k, torch.int32),
-                        ("head_map", head_map, torch.int32)):
-        _need_cuda(name, t, dt)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need_cuda(name, t, q.dtype)
+    _need_kv_like(k, v, B, N, d)
     k_max = idx.shape[-1]
+    n_tiles = N // TILE
+    _need_size("idx", idx, torch.int32, B * n_tiles * Hkv * k_max)
+    _need_size("idx_k", idx_k, torch.int32, B * n_tiles * Hkv)
+    _need_size("head_map", head_map, torch.int32, Hkv)
     dev = q.device
     out = torch.empty_like(q) if out is None else out
     lse = torch.empty(B, Hq, N, dtype=torch.float32, device=dev) if lse is None else lse
+    _need_size("out", out, q.dtype, q.numel())
+    _need_size("lse", lse, torch.float32, B * Hq * N)
     shape = Shape(B, Hq, Hkv, d)
     need = _lib().kascade_prefill_reuse_workspace_bytes(shape, N, k_max)
     ws = workspace(need, dev) if ws is None else ws
     rc = getattr(_lib(), "kascade_prefill_reuse" + sfx)(shape, int(N), _ptr(q), _ptr(k), _ptr(v), _ptr(idx),
                                       _ptr(idx_k), int(k_max), _ptr(head_map), float(scale),
-                                      _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream())
+                                      _ptr(out), _ptr(lse), _ptr(ws), _ws_bytes(ws), _stream())
     check(rc, "kascade_prefill_reuse" + sfx)
     return out, lse
 
@@ -266,16 +325,18 @@ def similarity_rows(p_b, row_len, row_k, idx_a, idx_b, b_row=None, a_row=None, o
     distribution p_b[b_row[r]] (identity maps when b_row / a_row are None).
     """
     _need_cuda("p_b", p_b, torch.float32)
-    for name, t in (("row_len", row_len), ("row_k", row_k), ("idx_a", idx_a), ("idx_b", idx_b)):
-        _need_cuda(name, t, torch.int32)
-    for name, t in (("b_row", b_row), ("a_row", a_row)):
-        if t is not None:
-            _need_cuda(name, t, torch.int32)
     ld = p_b.shape[-1]
     rows = p_b.numel() // ld if ld else 0
     k_max = idx_a.shape[-1]
+    for name, t, n in (("row_len", row_len, rows), ("row_k", row_k, rows),
+                       ("idx_a", idx_a, rows * k_max), ("idx_b", idx_b, rows * k_max)):
+        _need_size(name, t, torch.int32, n)
     n_out = b_row.numel() if b_row is not None else rows
+    for name, t in (("b_row", b_row), ("a_row", a_row)):
+        if t is not None:
+            _need_size(name, t, torch.int32, n_out)
     out = torch.empty(n_out, dtype=torch.float64, device=p_b.device) if out is None else out
+    _need_size("out", out, torch.float64, n_out)
     rc = _lib().kascade_similarity_rows(_ptr(p_b), int(rows), int(ld), _ptr(row_len), _ptr(row_k),
                                         _ptr(idx_a), _ptr(idx_b), int(k_max), int(n_out),
                                         _ptr(b_row), _ptr(a_row), _ptr(out), _stream())
