@@ -11,9 +11,12 @@
  *   [abstract]  the arXiv abstract (fugumt.com listing of 2512.16391v1).
  *
  * General rules (every entry point):
- *   - Every pointer argument is a DEVICE pointer owned by the caller; the library
- *     never allocates, frees or keeps a pointer after the call returns.  Scratch
- *     memory is passed in as `ws` of `ws_bytes` (query the size first).
+ *   - Every pointer argument is a DEVICE pointer owned by the caller (the host-side
+ *     calibration DP kascade_select_anchors excepted); the library never allocates,
+ *     frees or keeps a pointer after the call returns.  Scratch memory is passed in
+ *     as `ws` of `ws_bytes` (query the size first).  The one exception is
+ *     kascade_decode_anchor_static_ws, whose scratch is a fixed array owned by the
+ *     library (see its comment block).
  *   - bf16 tensors are passed as uint16_t bit patterns (IEEE bfloat16).
  *   - Every base pointer must be 16-byte aligned; every row stride named below is
  *     in elements and must keep rows 16-byte aligned.
@@ -24,7 +27,8 @@
  *     out of range, a NaN score) never fault: the offending element is skipped, and
  *     a sticky per-device status word is set; read it with kascade_get_device_status.
  *   - Supported shapes: head_dim d == 128, Hq % Hkv == 0, group size Hq/Hkv in {1,2,4,8},
- *     prefill query tile fixed at 128 tokens, prefill length a multiple of 128.
+ *     prefill query tile fixed at 128 tokens, prefill length a multiple of 128, decode
+ *     max_T and k_max at most 2^30 (KASCADE_ERR_UNSUPPORTED_SHAPE otherwise).
  *   - `scale` must be finite; the prefill calls also require scale > 0.
  *   - Returned status codes are the kascade_status values below; no C++ exception
  *     crosses this boundary.
@@ -103,13 +107,16 @@ int kascade_decode_anchor(kascade_shape s, const uint16_t* q, const uint16_t* k,
  * memory to its KV-cache pool up front (and cudaMalloc / cudaFree would also
  * synchronise the device in the middle of a step).
  *
- * Same arguments, results and checks as kascade_decode_anchor, minus ws/ws_bytes.
+ * Same arguments, results and checks as kascade_decode_anchor, minus ws/ws_bytes; the
+ * argument checks run first, in the same order, so a bad argument returns the same
+ * code as from kascade_decode_anchor; the scratch-size limit below is checked after them.
  * The scratch is a file-scope device array of KASCADE_STATIC_SCRATCH_BYTES that
  * every GPU which loads the library holds until the process exits.  The call
  * allocates nothing (no cudaMalloc, cudaFree or allocating library routine).
  *   - Problems whose scratch, kascade_decode_anchor_workspace_bytes(s, max_T), is
  *     larger than KASCADE_STATIC_SCRATCH_BYTES are refused with
- *     KASCADE_ERR_WORKSPACE_TOO_SMALL before anything is launched.
+ *     KASCADE_ERR_WORKSPACE_TOO_SMALL before anything is launched.  With 32 query
+ *     heads, 16 sequences of 4K tokens or one of 64K fit; one of 128K does not.
  *   - The first call on a device looks up the array's device address with
  *     cudaGetSymbolAddress (this may load the library's kernels on that device);
  *     make that first call before any stream capture.
@@ -235,7 +242,9 @@ int kascade_prefill_reuse_f16(kascade_shape s, int32_t N, const uint16_t* q, con
  * and (anchor) max_pages * page_size >= max_T.  A block-table entry outside
  * [0, num_pages) skips the tokens it holds and sets KASCADE_ERR_BAD_INDEX in the
  * device status; a sequence longer than max_pages * page_size is skipped the same
- * way.  Results are bit-identical to the contiguous calls on the same data. */
+ * way.  Results are bit-identical to the contiguous calls on the same data.
+ * The _f16 variants take fp16 q, k_pages, v_pages and out (same containers),
+ * like the contiguous _f16 calls. */
 int kascade_decode_anchor_paged(kascade_shape s, const uint16_t* q, const uint16_t* k_pages,
                                 const uint16_t* v_pages, int32_t num_pages,
                                 const int32_t* block_table, int32_t max_pages, int32_t page_size,
@@ -248,6 +257,18 @@ int kascade_decode_reuse_paged(kascade_shape s, const uint16_t* q, const uint16_
                                const int32_t* seq_len, const int32_t* idx, const int32_t* idx_k,
                                int32_t k_max, const int32_t* head_map, float scale, uint16_t* out,
                                float* lse, void* ws, size_t ws_bytes, void* stream);
+int kascade_decode_anchor_paged_f16(kascade_shape s, const uint16_t* q, const uint16_t* k_pages,
+                                    const uint16_t* v_pages, int32_t num_pages,
+                                    const int32_t* block_table, int32_t max_pages, int32_t page_size,
+                                    const int32_t* seq_len, int32_t max_T, float scale, uint16_t* out,
+                                    float* lse, float* pooled, int64_t ld_pooled, void* ws,
+                                    size_t ws_bytes, void* stream);
+int kascade_decode_reuse_paged_f16(kascade_shape s, const uint16_t* q, const uint16_t* k_pages,
+                                   const uint16_t* v_pages, int32_t num_pages,
+                                   const int32_t* block_table, int32_t max_pages, int32_t page_size,
+                                   const int32_t* seq_len, const int32_t* idx, const int32_t* idx_k,
+                                   int32_t k_max, const int32_t* head_map, float scale, uint16_t* out,
+                                   float* lse, void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------- */
 /* Calibration (Kascade explainer, レイヤー間類似度とアンカーレイヤー選択 and
@@ -274,6 +295,41 @@ int kascade_similarity_rows(const float* p_b, int32_t rows, int64_t ld, const in
                             const int32_t* row_k, const int32_t* idx_a, const int32_t* idx_b,
                             int32_t k_max, int32_t n_out, const int32_t* b_row,
                             const int32_t* a_row, double* ratio, void* stream);
+
+/* kascade_similarity_mean: sim(a, b) of two layers, the mean over the rows of the
+ * ratios kascade_similarity_rows defines (with identity row maps), summed in fp64
+ * in a fixed order.  The pages do not say how per-query ratios combine; the mean
+ * over queries (or pooled rows) is taken.
+ *   p_b, row_len, row_k, idx_a, idx_b, k_max  as in kascade_similarity_rows
+ *   mean      device fp64 [1]: output
+ *   ws        device scratch of kascade_similarity_mean_workspace_bytes(rows) bytes
+ * Errors as for kascade_similarity_rows; rows must be >= 1. */
+size_t kascade_similarity_mean_workspace_bytes(int32_t rows);
+int kascade_similarity_mean(const float* p_b, int32_t rows, int64_t ld, const int32_t* row_len,
+                            const int32_t* row_k, const int32_t* idx_a, const int32_t* idx_b,
+                            int32_t k_max, double* mean, void* ws, size_t ws_bytes, void* stream);
+
+/* kascade_head_remap: [explainer] ヘッドリマッピング.  For each key head h of a
+ * reuse layer, the anchor-layer key head whose Top-k indices recover the most of
+ * h's Top-k probability mass:
+ *     sim[h][a]   = mean over q < Q of ratio(p_reuse row h·Q+q; idx_anchor row a·Q+q,
+ *                                            idx_reuse row h·Q+q)
+ *     head_map[h] = argmax_a sim[h][a], the lowest a among equal maxima
+ * with ratio as in kascade_similarity_rows (a = anchor head, b = reuse head).
+ *   p_reuse     device fp32 [Hkv·Q, ld]: the reuse layer's distributions, row h·Q+q
+ *   row_len, row_k  device int32 [Hkv·Q]
+ *   idx_anchor  device int32 [Hkv·Q, k_max]: the anchor layer's Top-k rows
+ *   idx_reuse   device int32 [Hkv·Q, k_max]: the reuse layer's Top-k rows
+ *   sim         device fp64 [Hkv, Hkv]: output, or NULL
+ *   head_map    device int32 [Hkv]: output, values in [0, Hkv)
+ *   ws          device scratch of kascade_head_remap_workspace_bytes(Hkv, Q) bytes
+ * Returns KASCADE_ERR_INVALID_ARG unless 1 <= Hkv <= 1024, Q >= 1 and Hkv·Hkv·Q < 2^31;
+ * other errors as for kascade_similarity_rows.  Asynchronous on `stream`. */
+size_t kascade_head_remap_workspace_bytes(int32_t Hkv, int32_t Q);
+int kascade_head_remap(const float* p_reuse, int32_t Hkv, int32_t Q, int64_t ld, const int32_t* row_len,
+                       const int32_t* row_k, const int32_t* idx_anchor, const int32_t* idx_reuse,
+                       int32_t k_max, double* sim, int32_t* head_map, void* ws, size_t ws_bytes,
+                       void* stream);
 
 /* kascade_select_anchors: Algorithm 1 of the explainer on the HOST (no GPU
  * work).  S is host fp64 [L, L] row-major, the weighted similarity matrix

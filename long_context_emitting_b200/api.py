@@ -158,11 +158,12 @@ def decode_reuse(q, k, v, kv_off, seq_len, idx, idx_k, head_map, scale: float, H
 
 
 # ------------------------------------------------------------ decode, paged ----
-def _need_pages(k_pages, v_pages, block_table, B: int, Hkv: int, page_size: int, d: int) -> None:
+def _need_pages(k_pages, v_pages, block_table, B: int, Hkv: int, page_size: int, d: int,
+                dtype: torch.dtype = torch.bfloat16) -> None:
     """Page store [num_pages, Hkv, page_size, d] (K and V alike) and a block
     table with a row of page numbers for each of the B sequences."""
-    _need_cuda("k_pages", k_pages, torch.bfloat16)
-    _need_cuda("v_pages", v_pages, torch.bfloat16)
+    _need_cuda("k_pages", k_pages, dtype)
+    _need_cuda("v_pages", v_pages, dtype)
     _need_cuda("block_table", block_table, torch.int32)
     if k_pages.dim() != 4 or tuple(k_pages.shape[1:]) != (Hkv, page_size, d):
         raise ValueError(f"k_pages must be [num_pages, {Hkv}, {page_size}, {d}], got {tuple(k_pages.shape)}")
@@ -175,56 +176,60 @@ def _need_pages(k_pages, v_pages, block_table, B: int, Hkv: int, page_size: int,
 def decode_anchor_paged(q, k_pages, v_pages, block_table, page_size: int, seq_len, max_T: int,
                         scale: float, Hkv: int, out=None, lse=None, pooled=None,
                         ld_pooled: Optional[int] = None, ws=None):
-    """kascade_decode_anchor over a paged cache (see paging.to_paged)."""
+    """kascade_decode_anchor over a paged cache (see paging.to_paged); the _f16
+    entry point when q and the pages are float16."""
     B, Hq, d = q.shape
-    _need_cuda("q", q, torch.bfloat16)
-    _need_pages(k_pages, v_pages, block_table, B, Hkv, page_size, d)
+    sfx = _data_suffix(q, k_pages, v_pages)
+    _need_cuda("q", q, q.dtype)
+    _need_pages(k_pages, v_pages, block_table, B, Hkv, page_size, d, q.dtype)
     _need_size("seq_len", seq_len, torch.int32, B)
     dev = q.device
     if ld_pooled is None:
         ld_pooled = (max_T + 3) // 4 * 4
-    out = torch.empty(B, Hq, d, dtype=torch.bfloat16, device=dev) if out is None else out
+    out = torch.empty(B, Hq, d, dtype=q.dtype, device=dev) if out is None else out
     lse = torch.empty(B, Hq, dtype=torch.float32, device=dev) if lse is None else lse
     pooled = torch.empty(B, Hkv, ld_pooled, dtype=torch.float32, device=dev) if pooled is None else pooled
-    _need_size("out", out, torch.bfloat16, B * Hq * d)
+    _need_size("out", out, q.dtype, B * Hq * d)
     _need_size("lse", lse, torch.float32, B * Hq)
     _need_size("pooled", pooled, torch.float32, B * Hkv * ld_pooled)
     shape = Shape(B, Hq, Hkv, d)
     need = _lib().kascade_decode_anchor_workspace_bytes(shape, max_T)
     ws = workspace(need, dev) if ws is None else ws
-    rc = _lib().kascade_decode_anchor_paged(
+    rc = getattr(_lib(), "kascade_decode_anchor_paged" + sfx)(
         shape, _ptr(q), _ptr(k_pages), _ptr(v_pages), int(k_pages.shape[0]), _ptr(block_table),
         int(block_table.shape[1]), int(page_size), _ptr(seq_len), int(max_T), float(scale),
         _ptr(out), _ptr(lse), _ptr(pooled), int(ld_pooled), _ptr(ws), _ws_bytes(ws), _stream())
-    check(rc, "kascade_decode_anchor_paged")
+    check(rc, "kascade_decode_anchor_paged" + sfx)
     return out, lse, pooled
 
 
 def decode_reuse_paged(q, k_pages, v_pages, block_table, page_size: int, seq_len, idx, idx_k,
                        head_map, scale: float, Hkv: int, out=None, lse=None, ws=None):
-    """kascade_decode_reuse over a paged cache (see paging.to_paged)."""
+    """kascade_decode_reuse over a paged cache (see paging.to_paged); the _f16
+    entry point when q and the pages are float16."""
     B, Hq, d = q.shape
-    _need_cuda("q", q, torch.bfloat16)
-    _need_pages(k_pages, v_pages, block_table, B, Hkv, page_size, d)
+    sfx = _data_suffix(q, k_pages, v_pages)
+    _need_cuda("q", q, q.dtype)
+    _need_pages(k_pages, v_pages, block_table, B, Hkv, page_size, d, q.dtype)
     k_max = idx.shape[-1]
     _need_size("seq_len", seq_len, torch.int32, B)
     _need_size("idx", idx, torch.int32, B * Hkv * k_max)
     _need_size("idx_k", idx_k, torch.int32, B * Hkv)
     _need_size("head_map", head_map, torch.int32, Hkv)
     dev = q.device
-    out = torch.empty(B, Hq, d, dtype=torch.bfloat16, device=dev) if out is None else out
+    out = torch.empty(B, Hq, d, dtype=q.dtype, device=dev) if out is None else out
     lse = torch.empty(B, Hq, dtype=torch.float32, device=dev) if lse is None else lse
-    _need_size("out", out, torch.bfloat16, B * Hq * d)
+    _need_size("out", out, q.dtype, B * Hq * d)
     _need_size("lse", lse, torch.float32, B * Hq)
     shape = Shape(B, Hq, Hkv, d)
     need = _lib().kascade_decode_reuse_workspace_bytes(shape, k_max)
     ws = workspace(need, dev) if ws is None else ws
-    rc = _lib().kascade_decode_reuse_paged(
+    rc = getattr(_lib(), "kascade_decode_reuse_paged" + sfx)(
         shape, _ptr(q), _ptr(k_pages), _ptr(v_pages), int(k_pages.shape[0]), _ptr(block_table),
         int(block_table.shape[1]), int(page_size), _ptr(seq_len), _ptr(idx), _ptr(idx_k),
         int(k_max), _ptr(head_map), float(scale), _ptr(out), _ptr(lse), _ptr(ws), _ws_bytes(ws),
         _stream())
-    check(rc, "kascade_decode_reuse_paged")
+    check(rc, "kascade_decode_reuse_paged" + sfx)
     return out, lse
 
 
@@ -363,6 +368,27 @@ def _row_sets(p, k, n):
     return topk(p, row_len, row_k, k), row_len, row_k
 
 
+def similarity_mean(p_b, row_len, row_k, idx_a, idx_b, out=None, ws=None):
+    """sim(a, b) on the device (kascade_similarity_mean): fp64 [1], the mean over
+    rows of the per-row ratios of similarity_rows with identity row maps."""
+    _need_cuda("p_b", p_b, torch.float32)
+    ld = p_b.shape[-1]
+    rows = p_b.numel() // ld if ld else 0
+    k_max = idx_a.shape[-1]
+    for name, t, n in (("row_len", row_len, rows), ("row_k", row_k, rows),
+                       ("idx_a", idx_a, rows * k_max), ("idx_b", idx_b, rows * k_max)):
+        _need_size(name, t, torch.int32, n)
+    out = torch.empty(1, dtype=torch.float64, device=p_b.device) if out is None else out
+    _need_size("out", out, torch.float64, 1)
+    need = _lib().kascade_similarity_mean_workspace_bytes(int(rows))
+    ws = workspace(need, p_b.device) if ws is None else ws
+    rc = _lib().kascade_similarity_mean(_ptr(p_b), int(rows), int(ld), _ptr(row_len), _ptr(row_k),
+                                        _ptr(idx_a), _ptr(idx_b), int(k_max), _ptr(out), _ptr(ws),
+                                        _ws_bytes(ws), _stream())
+    check(rc, "kascade_similarity_mean")
+    return out
+
+
 def similarity(p_a, p_b, k: int) -> float:
     """sim(a, b) of two layers: the mean over rows (queries, or pooled rows) of
     the share of b's Top-k mass that a's Top-k indices recover."""
@@ -370,7 +396,7 @@ def similarity(p_a, p_b, k: int) -> float:
     p_a, p_b = _pad4(p_a), _pad4(p_b)
     ia, row_len, row_k = _row_sets(p_a, k, n)
     ib, _, _ = _row_sets(p_b, k, n)
-    return float(similarity_rows(p_b, row_len, row_k, ia, ib).mean().item())
+    return float(similarity_mean(p_b, row_len, row_k, ia, ib).item())
 
 
 def similarity_matrix(p_layers, k: int):
@@ -378,22 +404,24 @@ def similarity_matrix(p_layers, k: int):
     per-layer distributions p_layers [L, rows, n] (one Top-k pass per layer)."""
     L, n = p_layers.shape[0], p_layers.shape[-1]
     p_layers = _pad4(p_layers)
+    dev = p_layers.device
     sets = [_row_sets(p_layers[l], k, n) for l in range(L)]
-    sim = torch.zeros(L, L, dtype=torch.float64)
+    sim = torch.zeros(L, L, dtype=torch.float64, device=dev)
+    ws = workspace(_lib().kascade_similarity_mean_workspace_bytes(int(p_layers.shape[1])), dev)
     for a in range(L):
         for b in range(a, L):
             ib, row_len, row_k = sets[b]
-            r = similarity_rows(p_layers[b], row_len, row_k, sets[a][0], ib)
-            sim[a, b] = r.mean().item()
-    return sim.numpy()
+            similarity_mean(p_layers[b], row_len, row_k, sets[a][0], ib, out=sim[a, b:b + 1], ws=ws)
+    return sim.cpu().numpy()
 
 
-def head_remap(p_anchor, p_reuse, k: int):
-    """Reuse-layer KV head -> anchor KV head with the highest similarity.
+def head_remap(p_anchor, p_reuse, k: int, sim=None):
+    """Reuse-layer KV head -> anchor KV head with the highest similarity
+    (kascade_head_remap; ties go to the lower anchor head).
 
-    p_anchor / p_reuse: [Hkv, Q, n] distributions.  One similarity launch covers
-    every (reuse head, anchor head) pair; ties go to the lower anchor head.
-    Returns int64 [Hkv] on the device.
+    p_anchor / p_reuse: [Hkv, Q, n] distributions.  Returns int32 [Hkv] on the
+    device; ``sim`` (fp64 [Hkv, Hkv] on the device), when given, receives the
+    mean similarity of every (reuse head, anchor head) pair.
     """
     Hkv, Q, n = p_anchor.shape
     p_anchor, p_reuse = _pad4(p_anchor), _pad4(p_reuse)
@@ -401,13 +429,15 @@ def head_remap(p_anchor, p_reuse, k: int):
     ia, row_len, row_k = _row_sets(p_anchor.reshape(Hkv * Q, ld), k, n)
     ib, _, _ = _row_sets(p_reuse.reshape(Hkv * Q, ld), k, n)
     dev = p_anchor.device
-    h = torch.arange(Hkv, device=dev).view(Hkv, 1, 1)
-    a = torch.arange(Hkv, device=dev).view(1, Hkv, 1)
-    q = torch.arange(Q, device=dev).view(1, 1, Q)
-    b_row = (h * Q + q).expand(Hkv, Hkv, Q).reshape(-1).to(torch.int32).contiguous()
-    a_row = (a * Q + q).expand(Hkv, Hkv, Q).reshape(-1).to(torch.int32).contiguous()
-    r = similarity_rows(p_reuse.reshape(Hkv * Q, ld), row_len, row_k, ia, ib, b_row, a_row)
-    return r.view(Hkv, Hkv, Q).mean(-1).argmax(dim=1)
+    if sim is not None:
+        _need_size("sim", sim, torch.float64, Hkv * Hkv)
+    head_map = torch.empty(Hkv, dtype=torch.int32, device=dev)
+    ws = workspace(_lib().kascade_head_remap_workspace_bytes(int(Hkv), int(Q)), dev)
+    rc = _lib().kascade_head_remap(_ptr(p_reuse.reshape(Hkv * Q, ld)), int(Hkv), int(Q), int(ld),
+                                   _ptr(row_len), _ptr(row_k), _ptr(ia), _ptr(ib), int(k),
+                                   _ptr(sim), _ptr(head_map), _ptr(ws), _ws_bytes(ws), _stream())
+    check(rc, "kascade_head_remap")
+    return head_map
 
 
 def select_anchors(S, M: int):

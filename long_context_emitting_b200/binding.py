@@ -46,7 +46,13 @@ EXPORTS = (
     "kascade_prefill_reuse_f16",
     "kascade_decode_anchor_paged",
     "kascade_decode_reuse_paged",
+    "kascade_decode_anchor_paged_f16",
+    "kascade_decode_reuse_paged_f16",
     "kascade_similarity_rows",
+    "kascade_similarity_mean_workspace_bytes",
+    "kascade_similarity_mean",
+    "kascade_head_remap_workspace_bytes",
+    "kascade_head_remap",
     "kascade_select_anchors",
     "kascade_get_device_status",
     "kascade_status_string",
@@ -95,6 +101,12 @@ _SIGNATURES = {
                                                   _P, _I32, _P, _F, _P, _P, _P, _SZ, _P]),
     "kascade_similarity_rows": (ctypes.c_int, [_P, _I32, _I64, _P, _P, _P, _P, _I32, _I32, _P, _P,
                                                _P, _P]),
+    "kascade_similarity_mean_workspace_bytes": (_SZ, [_I32]),
+    "kascade_similarity_mean": (ctypes.c_int, [_P, _I32, _I64, _P, _P, _P, _P, _I32, _P, _P, _SZ,
+                                               _P]),
+    "kascade_head_remap_workspace_bytes": (_SZ, [_I32, _I32]),
+    "kascade_head_remap": (ctypes.c_int, [_P, _I32, _I32, _I64, _P, _P, _P, _P, _I32, _P, _P, _P,
+                                          _SZ, _P]),
     "kascade_select_anchors": (ctypes.c_int, [_P, _I32, _I32, _P, _P]),
     "kascade_get_device_status": (ctypes.c_int, [_P]),
     "kascade_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -102,7 +114,7 @@ _SIGNATURES = {
 }
 # fp16 variants take the same arguments as their bfloat16 counterparts
 for _name in ("kascade_decode_anchor", "kascade_decode_reuse", "kascade_prefill_anchor",
-              "kascade_prefill_reuse"):
+              "kascade_prefill_reuse", "kascade_decode_anchor_paged", "kascade_decode_reuse_paged"):
     _SIGNATURES[_name + "_f16"] = _SIGNATURES[_name]
 
 _lib = None

@@ -58,6 +58,11 @@ bool decode_logits_too_large(const kascade_shape& s, int32_t max_T) {
   return heads != 0 && (uint64_t)max_T > (1ull << 46) / heads;
 }
 
+// Per-row lengths (max_T, k_max) above 2^30 are refused: the kernels index a
+// row's tokens with 32-bit integers and round split sizes up, which must not
+// overflow (a 2^30-token row is already 512 GiB of K/V per key head).
+constexpr int32_t kMaxRowLen = 1 << 30;
+
 }  // namespace
 
 extern "C" {
@@ -103,25 +108,43 @@ int kascade_selftest_wait_timeout(int32_t spin, void* stream) {
 
 // ------------------------------------------------------------------ decode --
 size_t kascade_decode_anchor_workspace_bytes(kascade_shape s, int32_t max_T) {
-  if (check_shape(s) != KASCADE_OK || max_T < 0 || decode_logits_too_large(s, max_T)) return 0;
+  if (check_shape(s) != KASCADE_OK || max_T < 0 || max_T > kMaxRowLen || decode_logits_too_large(s, max_T))
+    return 0;
   return decode_workspace_bytes(s.B, s.Hkv, s.Hq / s.Hkv, max_T, true);
 }
+
+}  // extern "C"
+
+// Every host check of the decode anchor except the workspace ones, in the
+// order the entry points apply them (also used by the static-scratch entry).
+int kascade::decode_anchor_check_args(kascade_shape s, const uint16_t* q, const uint16_t* k,
+                                      const uint16_t* v, const int64_t* kv_off,
+                                      const int32_t* seq_len, int32_t max_T, float scale,
+                                      const uint16_t* out, const float* lse, const float* pooled,
+                                      int64_t ld_pooled) {
+  int rc = check_shape(s);
+  if (rc) return rc;
+  if (max_T < 0 || ld_pooled < max_T || (ld_pooled & 3) || !std::isfinite(scale))
+    return KASCADE_ERR_INVALID_ARG;
+  if (max_T > kMaxRowLen || decode_logits_too_large(s, max_T)) return KASCADE_ERR_UNSUPPORTED_SHAPE;
+  if (s.B == 0) return KASCADE_OK;
+  if (!q || !k || !v || !kv_off || !seq_len || !out || !pooled) return KASCADE_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(pooled) ||
+      (lse && !aligned16(lse)) || ((uintptr_t)kv_off & 7) || ((uintptr_t)seq_len & 3))
+    return KASCADE_ERR_INVALID_ARG;
+  return KASCADE_OK;
+}
+
+extern "C" {
 
 static int kascade_decode_anchor_impl(kascade_shape s, const uint16_t* q, const uint16_t* k,
                           const uint16_t* v, const int64_t* kv_off, const int32_t* seq_len,
                           int32_t max_T, float scale, uint16_t* out, float* lse,
                           float* pooled, int64_t ld_pooled, void* ws, size_t ws_bytes,
                           void* stream, bool f16) {
-  int rc = check_shape(s);
-  if (rc) return rc;
-  if (max_T < 0 || ld_pooled < max_T || (ld_pooled & 3) || !std::isfinite(scale))
-    return KASCADE_ERR_INVALID_ARG;
-  if (decode_logits_too_large(s, max_T)) return KASCADE_ERR_UNSUPPORTED_SHAPE;
-  if (s.B == 0) return KASCADE_OK;
-  if (!q || !k || !v || !kv_off || !seq_len || !out || !pooled || !ws) return KASCADE_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(pooled) ||
-      !aligned16(ws) || (lse && !aligned16(lse)) || ((uintptr_t)kv_off & 7) || ((uintptr_t)seq_len & 3))
-    return KASCADE_ERR_INVALID_ARG;
+  int rc = decode_anchor_check_args(s, q, k, v, kv_off, seq_len, max_T, scale, out, lse, pooled, ld_pooled);
+  if (rc || s.B == 0) return rc;
+  if (!ws || !aligned16(ws)) return KASCADE_ERR_INVALID_ARG;
   if (ws_bytes < kascade_decode_anchor_workspace_bytes(s, max_T)) return KASCADE_ERR_WORKSPACE_TOO_SMALL;
   DecodeParams p = {};
   p.f16 = f16;
@@ -151,7 +174,7 @@ int kascade_decode_anchor_f16(kascade_shape s, const uint16_t* q, const uint16_t
 }
 
 size_t kascade_decode_reuse_workspace_bytes(kascade_shape s, int32_t k_max) {
-  if (check_shape(s) != KASCADE_OK || k_max < 0) return 0;
+  if (check_shape(s) != KASCADE_OK || k_max < 0 || k_max > kMaxRowLen) return 0;
   return decode_workspace_bytes(s.B, s.Hkv, s.Hq / s.Hkv, k_max, false);
 }
 
@@ -163,6 +186,7 @@ static int kascade_decode_reuse_impl(kascade_shape s, const uint16_t* q, const u
   int rc = check_shape(s);
   if (rc) return rc;
   if (k_max < 0 || !std::isfinite(scale)) return KASCADE_ERR_INVALID_ARG;
+  if (k_max > kMaxRowLen) return KASCADE_ERR_UNSUPPORTED_SHAPE;
   if (s.B == 0) return KASCADE_OK;
   const size_t need = kascade_decode_reuse_workspace_bytes(s, k_max);
   if (!q || !k || !v || !kv_off || !seq_len || !idx || !idx_k || !head_map || !out || (need && !ws))
@@ -210,17 +234,17 @@ static int check_pages(const uint16_t* k, const uint16_t* v, const int32_t* bloc
   return KASCADE_OK;
 }
 
-int kascade_decode_anchor_paged(kascade_shape s, const uint16_t* q, const uint16_t* k_pages,
+static int kascade_decode_anchor_paged_impl(kascade_shape s, const uint16_t* q, const uint16_t* k_pages,
                                 const uint16_t* v_pages, int32_t num_pages,
                                 const int32_t* block_table, int32_t max_pages, int32_t page_size,
                                 const int32_t* seq_len, int32_t max_T, float scale, uint16_t* out,
                                 float* lse, float* pooled, int64_t ld_pooled, void* ws,
-                                size_t ws_bytes, void* stream) {
+                                size_t ws_bytes, void* stream, bool f16) {
   int rc = check_shape(s);
   if (rc) return rc;
   if (max_T < 0 || ld_pooled < max_T || (ld_pooled & 3) || !std::isfinite(scale))
     return KASCADE_ERR_INVALID_ARG;
-  if (decode_logits_too_large(s, max_T)) return KASCADE_ERR_UNSUPPORTED_SHAPE;
+  if (max_T > kMaxRowLen || decode_logits_too_large(s, max_T)) return KASCADE_ERR_UNSUPPORTED_SHAPE;
   if (s.B == 0) return KASCADE_OK;
   if ((rc = check_pages(k_pages, v_pages, block_table, num_pages, max_pages, page_size))) return rc;
   if ((int64_t)max_pages * page_size < max_T) return KASCADE_ERR_INVALID_ARG;
@@ -230,6 +254,7 @@ int kascade_decode_anchor_paged(kascade_shape s, const uint16_t* q, const uint16
     return KASCADE_ERR_INVALID_ARG;
   if (ws_bytes < kascade_decode_anchor_workspace_bytes(s, max_T)) return KASCADE_ERR_WORKSPACE_TOO_SMALL;
   DecodeParams p = {};
+  p.f16 = f16;
   p.B = s.B; p.Hq = s.Hq; p.Hkv = s.Hkv; p.G = s.Hq / s.Hkv;
   p.q = q; p.k = k_pages; p.v = v_pages; p.seq_len = seq_len; p.max_T = max_T;
   p.block_table = block_table; p.max_pages = max_pages; p.page_size = page_size;
@@ -241,15 +266,38 @@ int kascade_decode_anchor_paged(kascade_shape s, const uint16_t* q, const uint16
   return from_cuda(launch_decode_anchor(p, static_cast<cudaStream_t>(stream)));
 }
 
-int kascade_decode_reuse_paged(kascade_shape s, const uint16_t* q, const uint16_t* k_pages,
+int kascade_decode_anchor_paged(kascade_shape s, const uint16_t* q, const uint16_t* k_pages,
+                                const uint16_t* v_pages, int32_t num_pages,
+                                const int32_t* block_table, int32_t max_pages, int32_t page_size,
+                                const int32_t* seq_len, int32_t max_T, float scale, uint16_t* out,
+                                float* lse, float* pooled, int64_t ld_pooled, void* ws,
+                                size_t ws_bytes, void* stream) {
+  return kascade_decode_anchor_paged_impl(s, q, k_pages, v_pages, num_pages, block_table, max_pages, page_size,
+                                          seq_len, max_T, scale, out, lse, pooled, ld_pooled, ws, ws_bytes,
+                                          stream, false);
+}
+
+int kascade_decode_anchor_paged_f16(kascade_shape s, const uint16_t* q, const uint16_t* k_pages,
+                                    const uint16_t* v_pages, int32_t num_pages,
+                                    const int32_t* block_table, int32_t max_pages, int32_t page_size,
+                                    const int32_t* seq_len, int32_t max_T, float scale, uint16_t* out,
+                                    float* lse, float* pooled, int64_t ld_pooled, void* ws,
+                                    size_t ws_bytes, void* stream) {
+  return kascade_decode_anchor_paged_impl(s, q, k_pages, v_pages, num_pages, block_table, max_pages, page_size,
+                                          seq_len, max_T, scale, out, lse, pooled, ld_pooled, ws, ws_bytes,
+                                          stream, true);
+}
+
+static int kascade_decode_reuse_paged_impl(kascade_shape s, const uint16_t* q, const uint16_t* k_pages,
                                const uint16_t* v_pages, int32_t num_pages,
                                const int32_t* block_table, int32_t max_pages, int32_t page_size,
                                const int32_t* seq_len, const int32_t* idx, const int32_t* idx_k,
                                int32_t k_max, const int32_t* head_map, float scale, uint16_t* out,
-                               float* lse, void* ws, size_t ws_bytes, void* stream) {
+                               float* lse, void* ws, size_t ws_bytes, void* stream, bool f16) {
   int rc = check_shape(s);
   if (rc) return rc;
   if (k_max < 0 || !std::isfinite(scale)) return KASCADE_ERR_INVALID_ARG;
+  if (k_max > kMaxRowLen) return KASCADE_ERR_UNSUPPORTED_SHAPE;
   if (s.B == 0) return KASCADE_OK;
   if ((rc = check_pages(k_pages, v_pages, block_table, num_pages, max_pages, page_size))) return rc;
   const size_t need = kascade_decode_reuse_workspace_bytes(s, k_max);
@@ -261,6 +309,7 @@ int kascade_decode_reuse_paged(kascade_shape s, const uint16_t* q, const uint16_
     return KASCADE_ERR_INVALID_ARG;
   if (ws_bytes < need) return KASCADE_ERR_WORKSPACE_TOO_SMALL;
   DecodeParams p = {};
+  p.f16 = f16;
   p.B = s.B; p.Hq = s.Hq; p.Hkv = s.Hkv; p.G = s.Hq / s.Hkv;
   p.q = q; p.k = k_pages; p.v = v_pages; p.seq_len = seq_len;
   p.block_table = block_table; p.max_pages = max_pages; p.page_size = page_size;
@@ -273,6 +322,28 @@ int kascade_decode_reuse_paged(kascade_shape s, const uint16_t* q, const uint16_
   p.status = device_status_ptr();
   if (!p.status) return KASCADE_ERR_CUDA;
   return from_cuda(launch_decode_reuse(p, static_cast<cudaStream_t>(stream)));
+}
+
+int kascade_decode_reuse_paged(kascade_shape s, const uint16_t* q, const uint16_t* k_pages,
+                               const uint16_t* v_pages, int32_t num_pages,
+                               const int32_t* block_table, int32_t max_pages, int32_t page_size,
+                               const int32_t* seq_len, const int32_t* idx, const int32_t* idx_k,
+                               int32_t k_max, const int32_t* head_map, float scale, uint16_t* out,
+                               float* lse, void* ws, size_t ws_bytes, void* stream) {
+  return kascade_decode_reuse_paged_impl(s, q, k_pages, v_pages, num_pages, block_table, max_pages, page_size,
+                                         seq_len, idx, idx_k, k_max, head_map, scale, out, lse, ws, ws_bytes,
+                                         stream, false);
+}
+
+int kascade_decode_reuse_paged_f16(kascade_shape s, const uint16_t* q, const uint16_t* k_pages,
+                                   const uint16_t* v_pages, int32_t num_pages,
+                                   const int32_t* block_table, int32_t max_pages, int32_t page_size,
+                                   const int32_t* seq_len, const int32_t* idx, const int32_t* idx_k,
+                                   int32_t k_max, const int32_t* head_map, float scale, uint16_t* out,
+                                   float* lse, void* ws, size_t ws_bytes, void* stream) {
+  return kascade_decode_reuse_paged_impl(s, q, k_pages, v_pages, num_pages, block_table, max_pages, page_size,
+                                         seq_len, idx, idx_k, k_max, head_map, scale, out, lse, ws, ws_bytes,
+                                         stream, true);
 }
 
 // -------------------------------------------------------------------- topk --
@@ -319,6 +390,70 @@ int kascade_similarity_rows(const float* p_b, int32_t rows, int64_t ld, const in
   a.idx_a = idx_a; a.idx_b = idx_b; a.k_max = k_max; a.b_row = b_row; a.a_row = a_row;
   a.ratio = ratio; a.status = st;
   return from_cuda(launch_similarity_rows(a, n_out, static_cast<cudaStream_t>(stream)));
+}
+
+// Checks shared by the aggregating calibration calls: rows of p_b / row_len /
+// row_k / idx_a / idx_b as in kascade_similarity_rows.
+static int check_sim_rows(const float* p_b, int32_t rows, int64_t ld, const int32_t* row_len,
+                          const int32_t* row_k, const int32_t* idx_a, const int32_t* idx_b,
+                          int32_t k_max) {
+  if (rows <= 0 || ld < 0 || k_max < 0) return KASCADE_ERR_INVALID_ARG;
+  if (!p_b || !row_len || !row_k || (k_max > 0 && (!idx_a || !idx_b))) return KASCADE_ERR_INVALID_ARG;
+  if (!aligned16(p_b) || (ld & 3) || ((uintptr_t)row_len & 3) || ((uintptr_t)row_k & 3) ||
+      ((uintptr_t)idx_a & 3) || ((uintptr_t)idx_b & 3))
+    return KASCADE_ERR_INVALID_ARG;
+  return KASCADE_OK;
+}
+
+size_t kascade_similarity_mean_workspace_bytes(int32_t rows) {
+  return rows > 0 ? align_up((size_t)rows * sizeof(double), 256) : 0;
+}
+
+int kascade_similarity_mean(const float* p_b, int32_t rows, int64_t ld, const int32_t* row_len,
+                            const int32_t* row_k, const int32_t* idx_a, const int32_t* idx_b,
+                            int32_t k_max, double* mean, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_sim_rows(p_b, rows, ld, row_len, row_k, idx_a, idx_b, k_max);
+  if (rc) return rc;
+  if (!mean || ((uintptr_t)mean & 7) || !ws || ((uintptr_t)ws & 7)) return KASCADE_ERR_INVALID_ARG;
+  if (ws_bytes < kascade_similarity_mean_workspace_bytes(rows)) return KASCADE_ERR_WORKSPACE_TOO_SMALL;
+  unsigned* st = device_status_ptr();
+  if (!st) return KASCADE_ERR_CUDA;
+  SimArgs a;
+  a.p_b = p_b; a.rows = rows; a.ld = ld; a.row_len = row_len; a.row_k = row_k;
+  a.idx_a = idx_a; a.idx_b = idx_b; a.k_max = k_max; a.b_row = nullptr; a.a_row = nullptr;
+  a.ratio = nullptr; a.status = st;
+  return from_cuda(launch_similarity_mean(a, static_cast<double*>(ws), mean, static_cast<cudaStream_t>(stream)));
+}
+
+size_t kascade_head_remap_workspace_bytes(int32_t Hkv, int32_t Q) {
+  if (Hkv <= 0 || Hkv > 1024 || Q <= 0) return 0;
+  const size_t pairs = (size_t)Hkv * Hkv;
+  return align_up(pairs * Q * sizeof(double), 256) + align_up(pairs * sizeof(double), 256);
+}
+
+int kascade_head_remap(const float* p_reuse, int32_t Hkv, int32_t Q, int64_t ld, const int32_t* row_len,
+                       const int32_t* row_k, const int32_t* idx_anchor, const int32_t* idx_reuse,
+                       int32_t k_max, double* sim, int32_t* head_map, void* ws, size_t ws_bytes,
+                       void* stream) {
+  if (Hkv <= 0 || Hkv > 1024 || Q <= 0 || (int64_t)Hkv * Q > 0x7fffffff ||
+      (int64_t)Hkv * Hkv * Q > 0x7fffffff)
+    return KASCADE_ERR_INVALID_ARG;
+  int rc = check_sim_rows(p_reuse, Hkv * Q, ld, row_len, row_k, idx_anchor, idx_reuse, k_max);
+  if (rc) return rc;
+  if (!head_map || ((uintptr_t)head_map & 3) || (sim && ((uintptr_t)sim & 7)) || !ws || ((uintptr_t)ws & 7))
+    return KASCADE_ERR_INVALID_ARG;
+  if (ws_bytes < kascade_head_remap_workspace_bytes(Hkv, Q)) return KASCADE_ERR_WORKSPACE_TOO_SMALL;
+  unsigned* st = device_status_ptr();
+  if (!st) return KASCADE_ERR_CUDA;
+  const size_t pairs = (size_t)Hkv * Hkv;
+  double* ratio = static_cast<double*>(ws);
+  double* means = sim ? sim : reinterpret_cast<double*>(static_cast<char*>(ws) +
+                                                        align_up(pairs * Q * sizeof(double), 256));
+  SimArgs a;
+  a.p_b = p_reuse; a.rows = Hkv * Q; a.ld = ld; a.row_len = row_len; a.row_k = row_k;
+  a.idx_a = idx_anchor; a.idx_b = idx_reuse; a.k_max = k_max; a.b_row = nullptr; a.a_row = nullptr;
+  a.ratio = nullptr; a.status = st;
+  return from_cuda(launch_head_remap(a, Hkv, Q, ratio, means, head_map, static_cast<cudaStream_t>(stream)));
 }
 
 int kascade_select_anchors(const double* S, int32_t L, int32_t M, int32_t* anchors, double* best) {

@@ -7,11 +7,16 @@
 // maximising the covered weighted similarity, O(M L^2)).
 //
 // similarity_rows_kernel
-//   One CTA per output row r.  With rb = b_row[r] (or r) and ra = a_row[r] (or
+//   One CTA per output row r (head remap: one per (reuse head, anchor head,
+//   query row), the rows implied by the index arithmetic).  With rb = b_row[r] (or r) and ra = a_row[r] (or
 //   r) it sums, in fp64, P_b[rb, idx_a[ra, i]] and P_b[rb, idx_b[rb, i]] over
 //   i < k = row_k[rb], and writes their ratio.  The index lists are the Top-k
 //   outputs of layers a and b; indices outside [0, row_len[rb]) are skipped and
 //   flagged in the device status.
+// group_mean_kernel / remap_argmax_kernel
+//   The aggregation of the ratios: the mean over a layer's rows (sim(a, b)),
+//   and for the head remap the mean over queries of every head pair followed by
+//   the argmax over anchor heads, ties to the lower head (ヘッドリマッピング).
 #include "common.cuh"
 #include "internal.h"
 
@@ -27,8 +32,17 @@ constexpr int kSimThreads = 256;
 __global__ void __launch_bounds__(kSimThreads) similarity_rows_kernel(const SimArgs a) {
   __shared__ double s_num[kSimThreads / 32], s_den[kSimThreads / 32];
   const int r = blockIdx.x;
-  const int rb = a.b_row ? a.b_row[r] : r;
-  const int ra = a.a_row ? a.a_row[r] : r;
+  int rb, ra;
+  if (a.remap_Q > 0) {
+    // every (reuse head h, anchor head an, row q): r = (h * Hkv + an) * Q + q
+    const int Q = a.remap_Q, HQ = a.remap_H * a.remap_Q;
+    const int h = r / HQ, an = (r % HQ) / Q, q = r % Q;
+    rb = h * Q + q;
+    ra = an * Q + q;
+  } else {
+    rb = a.b_row ? a.b_row[r] : r;
+    ra = a.a_row ? a.a_row[r] : r;
+  }
   double num = 0.0, den = 0.0;
   bool bad = rb < 0 || rb >= a.rows || ra < 0 || ra >= a.rows;
   if (!bad) {
@@ -70,11 +84,71 @@ __global__ void __launch_bounds__(kSimThreads) similarity_rows_kernel(const SimA
   }
 }
 
+// Mean of each group of `len` consecutive ratios, in fp64 with a fixed
+// summation order (strided per-thread sums, then a fixed tree), one CTA per group.
+__global__ void __launch_bounds__(kSimThreads) group_mean_kernel(const double* ratio, int len, double* mean) {
+  __shared__ double s_sum[kSimThreads / 32];
+  const double* g = ratio + (int64_t)blockIdx.x * len;
+  double acc = 0.0;
+  for (int i = threadIdx.x; i < len; i += kSimThreads) acc += g[i];
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) s_sum[warp] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int w = 0; w < kSimThreads / 32; ++w) t += s_sum[w];
+    mean[blockIdx.x] = len > 0 ? t / (double)len : 0.0;
+  }
+}
+
+// head_map[h] = argmax over anchor heads a of sim[h][a], the lowest a among
+// equal maxima; one thread per reuse head.
+__global__ void remap_argmax_kernel(const double* sim, int Hkv, int32_t* head_map) {
+  const int h = threadIdx.x;
+  if (h >= Hkv) return;
+  int best = 0;
+  double bv = sim[(int64_t)h * Hkv];
+  for (int a = 1; a < Hkv; ++a) {
+    const double v = sim[(int64_t)h * Hkv + a];
+    if (v > bv) {
+      bv = v;
+      best = a;
+    }
+  }
+  head_map[h] = best;
+}
+
 }  // namespace
 
 cudaError_t launch_similarity_rows(const SimArgs& a, int n_out, cudaStream_t st) {
   if (n_out == 0) return cudaSuccess;
   similarity_rows_kernel<<<n_out, kSimThreads, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_similarity_mean(const SimArgs& a, double* ratio_ws, double* mean, cudaStream_t st) {
+  SimArgs r = a;
+  r.ratio = ratio_ws;
+  cudaError_t e = launch_similarity_rows(r, a.rows, st);
+  if (e != cudaSuccess) return e;
+  group_mean_kernel<<<1, kSimThreads, 0, st>>>(ratio_ws, a.rows, mean);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_head_remap(const SimArgs& a, int Hkv, int Q, double* ratio_ws, double* sim,
+                              int32_t* head_map, cudaStream_t st) {
+  SimArgs r = a;
+  r.ratio = ratio_ws;
+  r.remap_H = Hkv;
+  r.remap_Q = Q;
+  r.b_row = r.a_row = nullptr;
+  cudaError_t e = launch_similarity_rows(r, Hkv * Hkv * Q, st);
+  if (e != cudaSuccess) return e;
+  group_mean_kernel<<<Hkv * Hkv, kSimThreads, 0, st>>>(ratio_ws, Q, sim);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  remap_argmax_kernel<<<1, 32 * ((Hkv + 31) / 32), 0, st>>>(sim, Hkv, head_map);
   return cudaGetLastError();
 }
 

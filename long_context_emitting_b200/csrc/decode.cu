@@ -653,6 +653,10 @@ WsLayout ws_layout(int B, int Hkv, int G, int max_T, int nsplit, bool anchor) {
 
 }  // namespace
 
+// The split policy assumes B200's 148 SMs (here and in kSlots below) rather
+// than querying the device: the workspace query has no device argument, and
+// its size must equal what the launch uses.  On a part with another SM count
+// the results are the same, only the occupancy differs.
 #ifndef KASCADE_DECODE_TARGET_CTAS
 #define KASCADE_DECODE_TARGET_CTAS (4 * 148)
 #endif
@@ -670,10 +674,12 @@ DecodeSplit decode_split_for(int units, int n_items, bool gather) {
     constexpr int kSlots = 3 * 148;
     int nsplit = units >= kSlots ? 1 : kSlots / units;
     if (nsplit > 16) nsplit = 16;
-    int tpw = (n_items + 4 * nsplit - 1) / (4 * nsplit);
+    // 64-bit intermediates: n_items may be near the 2^30 row-length limit
+    int64_t tpw = ((int64_t)n_items + 4 * nsplit - 1) / (4 * nsplit);
     tpw = ((tpw + 15) / 16) * 16;
-    s.tok_per_warp = tpw > 16 ? tpw : 16;
-    s.nsplit = n_items > 0 ? (n_items + 4 * s.tok_per_warp - 1) / (4 * s.tok_per_warp) : 1;
+    s.tok_per_warp = (int)(tpw > 16 ? tpw : 16);
+    const int64_t per_cta = 4 * (int64_t)s.tok_per_warp;
+    s.nsplit = n_items > 0 ? (int)(((int64_t)n_items + per_cta - 1) / per_cta) : 1;
     return s;
   }
   // Largest per-warp run (<= KASCADE_DECODE_MAX_TPW items) that still gives at
@@ -685,13 +691,14 @@ DecodeSplit decode_split_for(int units, int n_items, bool gather) {
   constexpr int kTargetCtas = KASCADE_DECODE_TARGET_CTAS;
   int tpw = KASCADE_DECODE_MAX_TPW;
   while (tpw > 16) {
-    const int per_cta = kWarps * tpw;
-    const long long ctas = (long long)units * ((n_items + per_cta - 1) / per_cta);
+    const int64_t per_cta = (int64_t)kWarps * tpw;
+    const int64_t ctas = (int64_t)units * (((int64_t)n_items + per_cta - 1) / per_cta);
     if (ctas >= kTargetCtas) break;
     tpw /= 2;
   }
   s.tok_per_warp = tpw;
-  s.nsplit = n_items > 0 ? (n_items + kWarps * tpw - 1) / (kWarps * tpw) : 1;
+  const int64_t per_cta = (int64_t)kWarps * tpw;
+  s.nsplit = n_items > 0 ? (int)(((int64_t)n_items + per_cta - 1) / per_cta) : 1;
   return s;
 }
 

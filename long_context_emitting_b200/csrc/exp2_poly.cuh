@@ -4,7 +4,8 @@
 // obtained by adding and subtracting 1.5 * 2^23 (the sum's low mantissa bits
 // hold round(x)), so f lies in [-1/2, 1/2]; 2^f is a degree-5 minimax
 // polynomial for RELATIVE error on [-1/2, 1/2], computed for this library with
-// the Remez exchange algorithm and rounded to float; 2^n is applied by adding n
+// the Remez exchange algorithm (gen_exp2_poly.py beside this file prints the
+// coefficients) and rounded to float; 2^n is applied by adding n
 // to the exponent bits.  Valid for -125 <= x <= 0 after the clamp (smaller x
 // returns about 2^-125, which is zero next to a softmax sum >= 1).  Bound
 // checked in tests/test_exp2_poly.py (float32 evaluation, Horner with fused

@@ -6,6 +6,8 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "../../include/kascade.h"
+
 namespace kascade {
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -45,6 +47,10 @@ DecodeSplit decode_split_for(int units, int n_items, bool gather);
 size_t decode_workspace_bytes(int B, int Hkv, int G, int n_items, bool with_logits);
 
 cudaError_t launch_decode_anchor(const DecodeParams& p, cudaStream_t st);
+// Host checks of kascade_decode_anchor other than the workspace (api.cu).
+int decode_anchor_check_args(kascade_shape s, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                             const int64_t* kv_off, const int32_t* seq_len, int32_t max_T, float scale,
+                             const uint16_t* out, const float* lse, const float* pooled, int64_t ld_pooled);
 cudaError_t launch_decode_reuse(const DecodeParams& p, cudaStream_t st);
 
 // ------------------------------------------------------------------ topk ----
@@ -90,8 +96,15 @@ struct SimArgs {
   const int32_t* a_row;
   double* ratio;
   unsigned* status;
+  int remap_H = 0, remap_Q = 0;  // > 0: head-remap row arithmetic instead of b_row / a_row
 };
 cudaError_t launch_similarity_rows(const SimArgs& a, int n_out, cudaStream_t st);
+// Ratios of a.rows rows into ratio_ws, then their mean into *mean (device).
+cudaError_t launch_similarity_mean(const SimArgs& a, double* ratio_ws, double* mean, cudaStream_t st);
+// Ratios of every (reuse head, anchor head, query) into ratio_ws [Hkv*Hkv*Q],
+// their means over queries into sim [Hkv, Hkv], and the argmax into head_map.
+cudaError_t launch_head_remap(const SimArgs& a, int Hkv, int Q, double* ratio_ws, double* sim,
+                              int32_t* head_map, cudaStream_t st);
 
 // One CTA whose first thread waits on an mbarrier nothing arrives at, through
 // the prefill kernels' bounded wait (spin: the non-suspending variant); the

@@ -46,14 +46,13 @@ extern "C" int kascade_decode_anchor_static_ws(kascade_shape s, const uint16_t* 
                                                int32_t max_T, float scale, uint16_t* out,
                                                float* lse, float* pooled, int64_t ld_pooled,
                                                void* stream) {
-  // Size check first, so an oversized request is refused without touching CUDA.
+  // The regular entry point's argument checks come first, in its order, so a
+  // bad argument gets the same code from both; only then the size limit.
+  const int rc = kascade::decode_anchor_check_args(s, q, k, v, kv_off, seq_len, max_T, scale, out,
+                                                   lse, pooled, ld_pooled);
+  if (rc != KASCADE_OK || s.B == 0) return rc;
   const size_t need = kascade_decode_anchor_workspace_bytes(s, max_T);
   if (need > (size_t)KASCADE_STATIC_SCRATCH_BYTES) return KASCADE_ERR_WORKSPACE_TOO_SMALL;
-  // A bad shape (size 0) or an empty batch launches nothing: let the regular
-  // entry point report it without looking up the scratch array.
-  if (need == 0 || s.B == 0)
-    return kascade_decode_anchor(s, q, k, v, kv_off, seq_len, max_T, scale, out, lse, pooled,
-                                 ld_pooled, nullptr, 0, stream);
   void* ws = static_scratch_address();
   if (!ws) return KASCADE_ERR_CUDA;
   // Nothing in the scratch needs to start at zero: every partial and logit the

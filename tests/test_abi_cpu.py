@@ -115,3 +115,19 @@ def test_empty_batch_is_a_no_op(lib):
                                      16, None, 0, None) == OK
     assert lib.kascade_prefill_anchor(Shape(1, 32, 8, 128), 0, None, None, None, 0.1, None, None,
                                       None, None, 0, None) == OK
+
+
+def test_calibration_aggregates_check_arguments(lib):
+    # kascade_similarity_mean / kascade_head_remap refuse bad sizes and pointers on the host
+    INVALID, WS_SMALL = 1, 3
+    assert lib.kascade_similarity_mean_workspace_bytes(0) == 0
+    assert lib.kascade_similarity_mean_workspace_bytes(10) >= 80
+    assert lib.kascade_similarity_mean(P, 0, 64, P, P, P, P, 4, P, P, 1 << 20, None) == INVALID
+    assert lib.kascade_similarity_mean(P, 4, 63, P, P, P, P, 4, P, P, 1 << 20, None) == INVALID
+    assert lib.kascade_similarity_mean(P, 4, 64, P, P, P, P, 4, None, P, 1 << 20, None) == INVALID
+    assert lib.kascade_similarity_mean(P, 4, 64, P, P, P, P, 4, P, P, 8, None) == WS_SMALL
+    assert lib.kascade_head_remap_workspace_bytes(8, 16) >= 8 * 8 * 16 * 8
+    assert lib.kascade_head_remap_workspace_bytes(0, 16) == 0
+    assert lib.kascade_head_remap(P, 0, 16, 64, P, P, P, P, 4, P, P, P, 1 << 20, None) == INVALID
+    assert lib.kascade_head_remap(P, 8, 16, 64, P, P, P, P, 4, P, None, P, 1 << 20, None) == INVALID
+    assert lib.kascade_head_remap(P, 8, 16, 64, P, P, P, P, 4, P, P, P, 16, None) == WS_SMALL

@@ -41,10 +41,31 @@ def test_head_remap_matches_oracle():
         pa = _dirichlet(rng, (Hkv, Q, n), 0.3)
         perm = rng.permutation(Hkv)
         pr = pa[perm] * 0.9 + 0.1 * _dirichlet(rng, (Hkv, Q, n), 0.3)
-        got = api.head_remap(torch.from_numpy(pa).to(DEV), torch.from_numpy(pr).to(DEV), k)
+        sim = torch.full((Hkv, Hkv), float("nan"), dtype=torch.float64, device=DEV)
+        got = api.head_remap(torch.from_numpy(pa).to(DEV), torch.from_numpy(pr).to(DEV), k, sim=sim)
         ref = O.head_remap(pa.astype(np.float64), pr.astype(np.float64), k)
         assert got.cpu().tolist() == ref.tolist()
         assert ref.tolist() == perm.tolist()
+        # every pair's mean similarity (a = anchor head, b = reuse head)
+        sim_ref = np.array([[O.similarity(pa[a].astype(np.float64), pr[h].astype(np.float64), k)
+                             for a in range(Hkv)] for h in range(Hkv)])
+        assert np.abs(sim.cpu().numpy() - sim_ref).max() <= 1e-12
+    assert api.device_status() == 0
+
+
+def test_head_remap_ties_go_to_lower_anchor_head():
+    # anchor heads 1 and 3 are identical copies of reuse head 0's distribution, so
+    # both recover all of its mass; the lower one (1) must be chosen, as in the oracle
+    rng = np.random.default_rng(17)
+    Hkv, Q, n, k = 4, 5, 300, 30
+    pr = _dirichlet(rng, (Hkv, Q, n), 0.3)
+    pa = _dirichlet(rng, (Hkv, Q, n), 0.3)
+    pa[1] = pr[0]
+    pa[3] = pr[0]
+    got = api.head_remap(torch.from_numpy(pa).to(DEV), torch.from_numpy(pr).to(DEV), k)
+    ref = O.head_remap(pa.astype(np.float64), pr.astype(np.float64), k)
+    assert ref[0] == 1
+    assert got.cpu().tolist() == ref.tolist()
 
 
 def test_similarity_matrix_and_anchor_choice():

@@ -75,3 +75,13 @@ def test_packed_form_is_bit_identical():
         a = _exp2_poly(x, c)
         b = _exp2_poly_packed_form(x, c)
         assert a.view(np.uint32) == b.view(np.uint32), x
+
+
+def test_header_coefficients_come_from_the_generator():
+    # the Remez exchange generator beside the header reproduces its constants
+    from long_context_emitting_b200.csrc import gen_exp2_poly
+
+    got = gen_exp2_poly.float32_coefficients(5)
+    assert [float(c) for c in _coeffs("kExp2Deg5")] == got
+    _, err = gen_exp2_poly.remez_exp2(5)
+    assert err < 8e-8  # levelled relative error of the float64 polynomial
