@@ -142,6 +142,61 @@ def test_decode_b1_t4096_all_layers():
         assert_attention_close(_np(outs[l]), o_ref, f"layer {l}")
 
 
+def test_decode_b16_t32768_all_32_layers_sampled():
+    # The benchmark's whole decode step: 32 layers with anchors [0, 2, 8, 13, 14]
+    # and a per-layer drift of the planted directions, run layer by layer on the
+    # GPU for all 16 sequences and checked against the oracle's own schedule on
+    # two of them.  Every anchor's index sets are checked (a later anchor replaces
+    # the earlier one's), and every reuse layer against the oracle fed the GPU's
+    # current indices and, end to end, the oracle's own.
+    cfg = workload.DECODE_32K
+    lens = cfg.seq_lens()
+    seqs = [0, 11]
+    sch = DecodeSchedule(cfg.B, cfg.Hq, cfg.Hkv, lens, cfg.anchors, cfg.n_layers, DEV)
+    idx_ref = ks = None
+    n_anchor = 0
+    for l in range(cfg.n_layers):
+        inp = workload.decode_layer(cfg, l, DEV)
+        out = torch.empty(cfg.B, cfg.Hq, cfg.d, dtype=torch.bfloat16, device=DEV)
+        q = _np(inp["q"])[seqs]
+        kc, vc = _host_caches(cfg, inp, seqs)
+        slens = [lens[b] for b in seqs]
+        if sch.is_anchor(l):
+            n_anchor += 1
+            sch.run_anchor(inp, out)
+            sch.run_topk()
+            assert api.device_status() == 0
+            o_ref, _, pooled_ref = O.decode_anchor(q, kc, vc, slens, SCALE)
+            assert_attention_close(_np(out)[seqs], o_ref, f"layer {l} (anchor)")
+            idx_gpu = sch.idx.cpu().numpy()
+            k = O.k_for_len(cfg.T)
+            idx_ref = np.full((len(seqs), cfg.Hkv, sch.k_max), -1, dtype=np.int64)
+            for i, b in enumerate(seqs):
+                for h in range(cfg.Hkv):
+                    ref = O.topk_select(pooled_ref[i][h], k)
+                    idx_ref[i, h, :k] = ref
+                    assert_index_set_ok(idx_gpu[b, h], ref, pooled_ref[i][h], k, f"layer {l} b={b} h={h}")
+            ks = np.full((len(seqs), cfg.Hkv), k)
+        else:
+            hm = workload.head_map(cfg, l).to(DEV)
+            sch.run_reuse(inp, hm, out)
+            assert api.device_status() == 0
+            hm_np = hm.cpu().numpy()
+            idx_gpu = sch.idx.cpu().numpy()[seqs]
+            o_a, _ = O.decode_reuse(q, kc, vc, slens, idx_gpu, ks, hm_np, SCALE)
+            assert_attention_close(_np(out)[seqs], o_a, f"layer {l} (reuse, GPU indices)")
+            o_b, _ = O.decode_reuse(q, kc, vc, slens, idx_ref, ks, hm_np, SCALE)
+            assert_attention_close(_np(out)[seqs], o_b, f"layer {l} (reuse, oracle indices)")
+        del inp, out
+    assert n_anchor == 5
+
+
+def test_decode_b1_t524288():
+    # the longest decode context of the pages' speed table (512K tokens)
+    cfg = workload.scaled(workload.DECODE_4K, name="decode_b1_t524288", B=1, T=524288)
+    _check_layer_pair(cfg)
+
+
 def test_decode_b16_t32768_sampled():
     _check_layer_pair(workload.DECODE_32K, seqs=[0, 9, 15], reuse_layer=5)
 

@@ -45,38 +45,53 @@ def _check(cfg, tiles=None, reuse_layer=1, b=0, dtype=torch.bfloat16):
     sch.run_reuse(r_in, hm, out_r)
     assert api.device_status() == 0
 
+    # Only the sampled tiles' rows leave the GPU: pooled and index rows, outputs
+    # and LSE of the sampled query rows (the oracle only reads those tiles; its
+    # full-size index arrays are zero-initialised and filled for them alone).
+    rows = _rows(tiles)
+    rows_t = torch.from_numpy(rows).to(DEV)
+    got_a = _np(out_a[b].index_select(1, rows_t))
+    got_lse_a = _np(lse_a[b].index_select(1, rows_t))
+    got_r = _np(out_r[b].index_select(1, rows_t))
+    got_lse_r = _np(sch.lse[b].index_select(1, rows_t))
+    pooled_gpu = {t: sch.pooled[b, t].cpu().numpy() for t in tiles}
+    k_max = sch.k_max
+    idx_gpu = np.zeros((nt, cfg.Hkv, k_max), dtype=np.int64)
+    for t in tiles:
+        idx_gpu[t] = sch.idx[b, t].cpu().numpy()
+    del out_a, out_r, lse_a
+
     q, k, v = (_np(a_in[n][b]) for n in ("q", "k", "v"))
     o_ref, lse_ref, pooled_ref = O.prefill_anchor(q, k, v, SCALE, tile=TILE, tiles=tiles)
-    rows = _rows(tiles)
-    assert_attention_close(_np(out_a[b])[:, rows], o_ref[:, rows], "prefill anchor O")
-    np.testing.assert_allclose(_np(lse_a[b])[:, rows], lse_ref[:, rows], atol=LSE_ABS, rtol=0)
-    pooled_gpu = sch.pooled[b].cpu().numpy()
-    idx_gpu = sch.idx[b].cpu().numpy()
-    k_max = sch.k_max
-    idx_ref = np.full((nt, cfg.Hkv, k_max), -1, dtype=np.int64)
+    del q, k, v
+    assert_attention_close(got_a, o_ref[:, rows], "prefill anchor O")
+    np.testing.assert_allclose(got_lse_a, lse_ref[:, rows], atol=LSE_ABS, rtol=0)
+    del o_ref, lse_ref
+    idx_ref = np.zeros((nt, cfg.Hkv, k_max), dtype=np.int64)
     idx_k = np.zeros((nt, cfg.Hkv), dtype=np.int64)
     for t in tiles:
         P = TILE * t
         kt = O.k_for_len(P)
         idx_k[t] = kt
+        idx_ref[t] = -1
         for h in range(cfg.Hkv):
-            assert_pooled_close(pooled_gpu[t, h, :P], pooled_ref[t, h, :P], f"pooled t={t} h={h}")
-            exact = O.topk_select(pooled_gpu[t, h, :P].astype(np.float32), kt)
+            assert_pooled_close(pooled_gpu[t][h, :P], pooled_ref[t, h, :P], f"pooled t={t} h={h}")
+            exact = O.topk_select(pooled_gpu[t][h, :P].astype(np.float32), kt)
             assert np.array_equal(idx_gpu[t, h, :kt], exact), f"topk t={t} h={h}"
             assert (idx_gpu[t, h, kt:] == -1).all()
             ref = O.topk_select(pooled_ref[t, h, :P], kt)
             idx_ref[t, h, :kt] = ref
             assert_index_set_ok(idx_gpu[t, h], ref, pooled_ref[t, h, :P], kt, f"t={t} h={h}")
+    del pooled_ref
 
     hm_np = hm.cpu().numpy()
     qr, kr, vr = (_np(r_in[n][b]) for n in ("q", "k", "v"))
-    got = _np(out_r[b])[:, rows]
-    o_a, lse_ra = O.prefill_reuse(qr, kr, vr, idx_gpu.astype(np.int64), idx_k, hm_np, SCALE,
-                                  tile=TILE, tiles=tiles)
-    assert_attention_close(got, o_a[:, rows], "prefill reuse O (GPU indices)")
-    np.testing.assert_allclose(_np(sch.lse[b])[:, rows], lse_ra[:, rows], atol=LSE_ABS, rtol=0)
+    o_a, lse_ra = O.prefill_reuse(qr, kr, vr, idx_gpu, idx_k, hm_np, SCALE, tile=TILE, tiles=tiles)
+    assert_attention_close(got_r, o_a[:, rows], "prefill reuse O (GPU indices)")
+    np.testing.assert_allclose(got_lse_r, lse_ra[:, rows], atol=LSE_ABS, rtol=0)
+    del o_a, lse_ra
     o_b, _ = O.prefill_reuse(qr, kr, vr, idx_ref, idx_k, hm_np, SCALE, tile=TILE, tiles=tiles)
-    assert_attention_close(got, o_b[:, rows], "prefill reuse O (oracle indices)")
+    assert_attention_close(got_r, o_b[:, rows], "prefill reuse O (oracle indices)")
 
 
 def test_prefill_small_all_tiles():
@@ -124,6 +139,13 @@ def test_prefill_n65536_sampled_tiles():
 def test_prefill_n131072_sampled_tiles():
     cfg = workload.scaled(workload.PREFILL_64K, name="prefill_b1_n131072", N=131072)
     _check(cfg, tiles=[0, 3, 1023])
+
+
+def test_prefill_n262144_sampled_tiles():
+    # the longest prefill of the pages' speed table (256K tokens): the first,
+    # a middle and the last query tiles
+    cfg = workload.scaled(workload.PREFILL_64K, name="prefill_b1_n262144", N=262144)
+    _check(cfg, tiles=[0, 1, 1024, 2047])
 
 
 def test_prefill_reuse_full_prefix_is_dense():
