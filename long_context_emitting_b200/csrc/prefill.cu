@@ -7,7 +7,8 @@
 // 技術的詳細 › アンカーレイヤーと再利用レイヤー and › ヘッドリマッピング.
 //
 // prefill_attn_kernel<GATHER, F16>  (F16: fp16 data, else bf16)
-//   One CTA per (query tile t, pair of query heads of one GQA group, sequence).
+//   One CTA per (query tile t, pair of query heads of one GQA group, sequence),
+//   launched longest tiles first over the whole grid.
 //   The two heads share every K/V block, so each block is loaded once for two
 //   128 x 128 attention tiles.  Warp roles (384 threads, three warpgroups):
 //     warp 8      TMA producer: Q tiles, then K/V blocks into a 2-stage ring.
@@ -33,7 +34,7 @@
 //   TMEM (512 columns): S0|P0 [0,128), O0 [128,256), S1|P1 [256,384), O1 [384,512).
 //
 // prefill_pool_kernel
-//   One CTA per (tile t >= 1, KV head, sequence).  For each key block before
+//   One CTA per (tile t >= 1, KV head, sequence), longest tiles first.  For each key block before
 //   the tile it computes S^T = K Q_g^T for the group's query heads (keys on
 //   TMEM lanes, queries on columns, one 128-column TMEM tile per head), so a
 //   thread owns one key and sums exp2(s - lse2) over the tile's queries in
@@ -106,11 +107,11 @@ constexpr uint32_t kPoolQx = kPoolKx + kXBytes;         // [kPoolHeads] tiles
 constexpr uint32_t kPoolRed = kPoolQx + kPoolHeads * kXBytes;  // [2 slots][3 heads][128] floats
 constexpr uint32_t kPoolMisc = kPoolRed + 2 * 3 * kTile * 4;
 constexpr uint32_t kPoolSmem = kPoolMisc + 256 + 1024;
-// per head of the round: S^T tile full (MMA commit) / free (read into registers,
-// one arrival per warp); partial-sum exchange: heads 1-3 -> head 0's warpgroup
-// S / free per pair of heads (a single head when the group has one)
-enum { kPBarQ = 0, kPBarKFull = 1, kPBarKEmpty = 3, kPBarS = 5, kPBarFree = 9, kPBarRedFull = 13,
-       kPBarRedEmpty = 15, kPoolBars = 17 };
+// per TMEM buffer (two, alternating by sub-iteration): S^T full (MMA commit) /
+// free (read into registers, one arrival per warp); partial-sum exchange:
+// warpgroups 1.. -> warpgroup 0, double-buffered by block
+enum { kPBarQ = 0, kPBarKFull = 1, kPBarKEmpty = 3, kPBarS = 5, kPBarFree = 7, kPBarRedFull = 9,
+       kPBarRedEmpty = 11, kPoolBars = 13 };
 
 struct AttnArgs {
   int B, Hq, Hkv, G, N, n_tiles;
@@ -169,10 +170,23 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int t = a.n_tiles - 1 - (int)blockIdx.x;  // longest rows first
-  const int b = blockIdx.z;
+  // 1-D grid.  Anchor: longest tiles first over the whole grid (every head
+  // group and sequence of tile t before any of tile t - 1), so no long tile
+  // starts late.  Reuse: tiles longest first within each head group, the head
+  // groups one after another (the CTAs running together then gather from the
+  // same key head's rows, which measured faster than the global order).
   const int ntile = a.G >= 2 ? 2 : 1;
-  const int g0 = blockIdx.y * ntile;
+  const int HG = a.Hq / ntile;
+  int t, rem;
+  if (GATHER) {
+    t = a.n_tiles - 1 - (int)(blockIdx.x % a.n_tiles);
+    rem = (int)(blockIdx.x / a.n_tiles);
+  } else {
+    t = a.n_tiles - 1 - (int)(blockIdx.x / (HG * a.B));
+    rem = (int)(blockIdx.x % (HG * a.B));
+  }
+  const int g0 = (rem % HG) * ntile;
+  const int b = rem / HG;
   const int h = g0 / a.G;
 
   // ---- key blocks ------------------------------------------------------------
@@ -546,21 +560,26 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int t = a.n_tiles - 1 - (int)blockIdx.x;  // t >= 1, longest first
-  const int h = blockIdx.y, b = blockIdx.z;
+  // 1-D grid, longest tiles first over the whole grid (t >= 1)
+  const int per_t = a.Hkv * a.B;
+  const int t = a.n_tiles - 1 - (int)(blockIdx.x / per_t);
+  const int h = (int)(blockIdx.x % per_t) % a.Hkv, b = (int)(blockIdx.x % per_t) / a.Hkv;
   const int G = a.G;
   const int kv_row0 = (int)(((int64_t)b * a.Hkv + h) * a.N);
   const int n_rounds = (G + kPoolHeads - 1) / kPoolHeads;
   const int nblk = t;  // key blocks before the tile, per round
+  const int hg = G < kPoolHeads ? G : kPoolHeads;  // heads per round: 1, 2 or 4
+  const int n_sub = hg >= 2 ? hg / 2 : 1;         // head pairs per round
+  const int nwg = hg >= 2 ? 4 : 2;                // summing warpgroups in use
 
   if (tid == 0) {
     for (int i = 0; i < kPoolBars; ++i) {
-      // free: the head's 4 warps; exchange full: 12 warps of heads 1-3; empty: head 0's 4 warps
-      // free: the warps of the pair's (or single head's) warpgroups; exchange full:
-      // 12 warps of heads 1-3; exchange empty: head 0's 4 warps
-      const uint32_t n_free = G >= 2 ? 8u : 4u;
-      const uint32_t count = (i >= kPBarRedFull && i < kPBarRedEmpty) ? 12u
-                             : (i >= kPBarRedEmpty ? 4u : (i >= kPBarFree ? n_free : 1u));
+      // buffer free: every warp of the summing warpgroups in use; exchange full:
+      // the warps of warpgroups 1..; exchange empty: warpgroup 0's 4 warps
+      uint32_t count = 1;
+      if (i >= kPBarFree && i < kPBarFree + 2) count = 4u * nwg;
+      if (i >= kPBarRedFull && i < kPBarRedFull + 2) count = 4u * (nwg - 1);
+      if (i >= kPBarRedEmpty && i < kPBarRedEmpty + 2) count = 4u;
       mbar_init(bar(i), count);
     }
     *s_abort = 0;
@@ -604,12 +623,17 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   };
   // Each role runs its own copy of the round loop, so the compiler sizes every
   // role's code for that role's register budget (setmaxnreg below).
+  //
+  // Within a round, the key blocks are the outer loop and the round's head
+  // pairs ("sub-rounds") the inner one; sub-iteration it = (rd*nblk + jb)*n_sub
+  // + sub computes S^T of one head pair into TMEM buffer it & 1 (columns
+  // [256 (it&1), 256 (it&1) + 256): the pair's first head, then its second),
+  // so the MMA fills one buffer while the summing warps work on the other.
   if (warp < 4) {
     setmaxnreg_dec<kPoolCtlRegs>();
     for (int rd = 0; rd < n_rounds; ++rd) {
-      const int hg = min(kPoolHeads, G - rd * kPoolHeads);  // heads this round
       const int gbase = h * G + rd * kPoolHeads;
-      const int it0 = rd * nblk;  // running block counter for stage / phase bookkeeping
+      const int kit0 = rd * nblk;  // running K-block counter (stage / phase bookkeeping)
       load_lse(hg, gbase);
       if (warp == 0) {
         // ---------------------------- TMA producer ----------------------------
@@ -621,8 +645,8 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tma_load_2d(sbase + kPoolQ + (kPoolHeads + j) * kHalfBytes, &tm_q, 64, y, bar(kPBarQ));
           }
           for (int jb = 0; jb < nblk; ++jb) {
-            const int it = it0 + jb, st = it & 1;
-            if (it >= 2 && !mbar_wait(bar(kPBarKEmpty + st), ((it >> 1) - 1) & 1, a.status)) { *s_abort = 1; break; }
+            const int kit = kit0 + jb, st = kit & 1;
+            if (kit >= 2 && !mbar_wait(bar(kPBarKEmpty + st), ((kit >> 1) - 1) & 1, a.status)) { *s_abort = 1; break; }
             if (*s_abort) break;
             const uint32_t ks = sbase + kPoolK + st * kTileBytes;
             mbar_expect_tx(bar(kPBarKFull + st), kTileBytes);
@@ -632,30 +656,29 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
       } else if (warp == 1) {
         // ---------------------------- MMA issuer ------------------------------
-        // S^T = K [Q_g; Q_g+1]^T for each pair of heads of the round (N = 256; a
-        // single head uses N = 128) into TMEM columns 128 g .., as soon as both
-        // heads' summing warps have read the pair's previous tile.
+        // S^T = K [Q_g; Q_g+1]^T of each head pair (N = 256; a single head uses
+        // N = 128) into buffer it & 1, once the summing warps freed it.
         if (lane == 0) {
-          const int np = hg >= 2 ? hg / 2 : 1;
           // Q and K in the data's type; the extra -lse step below is a separate
           // instruction with bf16 operands on both sides
           const uint32_t idesc = idesc_f16kind(128, hg >= 2 ? 256 : 128, false, false, F16);
           const uint32_t idesc_x = idesc_bf16(128, hg >= 2 ? 256 : 128, false, false);
           bool ok = mbar_wait(bar(kPBarQ), rd & 1, a.status);
           for (int jb = 0; ok && jb < nblk; ++jb) {
-            const int it = it0 + jb, st = it & 1;
-            if (!(ok = mbar_wait(bar(kPBarKFull + st), (it >> 1) & 1, a.status))) break;
+            const int kit = kit0 + jb, st = kit & 1;
+            if (!(ok = mbar_wait(bar(kPBarKFull + st), (kit >> 1) & 1, a.status))) break;
             const uint64_t dk = kmajor_desc(sbase + kPoolK + st * kTileBytes, 0);
-            for (int pr = 0; pr < np; ++pr) {
-              if (it >= 1 && !(ok = mbar_spin(bar(kPBarFree + pr), (it - 1) & 1, a.status))) break;
+            for (int sub = 0; sub < n_sub; ++sub) {
+              const int it = kit * n_sub + sub, buf = it & 1;
+              if (it >= 2 && !(ok = mbar_spin(bar(kPBarFree + buf), ((it >> 1) - 1) & 1, a.status))) break;
               tc_fence_after();
-              const uint64_t dq = kmajor_desc(sbase + kPoolQ + 2 * pr * kHalfBytes, 0);
+              const uint64_t dq = kmajor_desc(sbase + kPoolQ + 2 * sub * kHalfBytes, 0);
 #pragma unroll
               for (int k16 = 0; k16 < 8; ++k16)
-                umma_ss(tmem + 256 * pr, dk + kmajor_step(k16), dq + qpair_step(k16), idesc, k16 > 0 ? 1u : 0u);
-              umma_ss(tmem + 256 * pr, sw32_desc(sbase + kPoolKx), sw32_desc(sbase + kPoolQx + 2 * pr * kXBytes),
+                umma_ss(tmem + 256 * buf, dk + kmajor_step(k16), dq + qpair_step(k16), idesc, k16 > 0 ? 1u : 0u);
+              umma_ss(tmem + 256 * buf, sw32_desc(sbase + kPoolKx), sw32_desc(sbase + kPoolQx + 2 * sub * kXBytes),
                       idesc_x, 1u);
-              umma_commit(bar(kPBarS + pr));
+              umma_commit(bar(kPBarS + buf));
             }
             if (!ok) break;
             umma_commit(bar(kPBarKEmpty + st));
@@ -668,29 +691,32 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     }
   } else {
     setmaxnreg_inc<kPoolSumRegs>();
-    // ------------------- summing warpgroups (one head each) -------------------
-    // Thread = key (TMEM lane).  The head's 128 scores are read 16 queries at
-    // a time, one load ahead of the summing; the tile is released to the MMA
-    // once the last columns are in registers, before they are summed.
-    const int g = (warp >> 2) - 1;  // head of the round handled by this warpgroup
+    // ------------------- summing warpgroups ---------------------------------
+    // Warpgroup w takes head (w >> 1) of each pair and query half (w & 1):
+    // thread = key (TMEM lane) sums exp2(sc (q.k - lse/scale)) over 64 queries
+    // of that head, read 16 at a time, one load ahead of the summing; the
+    // buffer is released once the last columns are in registers.
+    const int w = (warp >> 2) - 1;
+    const int hl = w >> 1, qh = w & 1;
+    const bool active = w < nwg;
     const int key = (warp & 3) * 32 + lane;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint64_t SC = f2_pack(a.scale_log2, a.scale_log2);
     for (int rd = 0; rd < n_rounds; ++rd) {
-      const int hg = min(kPoolHeads, G - rd * kPoolHeads);
       const int gbase = h * G + rd * kPoolHeads;
-      const int it0 = rd * nblk;
+      const int kit0 = rd * nblk;
       load_lse(hg, gbase);
-      float pend = 0.f;  // head 0's warpgroup: its own sum of the previous block
-      // adds heads 1-3 of block itp (block jbp of the round) to `mine`, writes pooled
-      auto combine = [&](int rdp, int itp, int jbp, float mine) -> bool {
-        const int sl = itp & 1;
-        if (!mbar_wait(bar(kPBarRedFull + sl), (itp >> 1) & 1, a.status)) {
+      float pend = 0.f;  // warpgroup 0: its own sum of the previous block
+      // adds warpgroups 1.. of block kitp (block jbp of the round) to `mine`, writes pooled
+      auto combine = [&](int rdp, int kitp, int jbp, float mine) -> bool {
+        const int sl = kitp & 1;
+        if (!mbar_wait(bar(kPBarRedFull + sl), (kitp >> 1) & 1, a.status)) {
           *s_abort = 1;
           return false;
         }
         const float* slot = red + sl * 3 * kTile;
-        const float tot = mine + slot[key] + slot[kTile + key] + slot[2 * kTile + key];
+        float tot = mine;
+        for (int o = 0; o < nwg - 1; ++o) tot += slot[o * kTile + key];
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(kPBarRedEmpty + sl));
         const int col = kTile * jbp + key;
@@ -699,7 +725,7 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         return true;
       };
       for (int jb = 0; jb < nblk; ++jb) {
-        const int it = it0 + jb;
+        const int kit = kit0 + jb;
         uint64_t A[4] = {0ull, 0ull, 0ull, 0ull};
         // sum over 16 queries of exp2(sc * (q.k - lse/scale)), two per packed
         // instruction; 2 of every 8 pairs on the FMA pipe, the rest on the SFU
@@ -718,60 +744,69 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             A[e2 & 3] = f2_add(A[e2 & 3], f2_pack(p0, p1));
           }
         };
-        if (g < hg) {
-          if (!mbar_wait(bar(kPBarS + g / 2), it & 1, a.status) || *s_abort) {
-            *s_abort = 1;
-            break;
-          }
-          tc_fence_after();
-          // The head's 128 scores in eight loads of 16 columns: each load is in
-          // flight while the previous columns are summed (a wait covers every
-          // earlier load; the fence keeps the compiler from reading a register
-          // before it).  The tile goes back to the MMA once the last load landed.
-          const uint32_t tS = tmem + 128 * g + lane_base;
-          uint32_t v0[16], v1[16];
-          tmem_ld16(tS, v0);
-          tmem_wait_ld();
-          reg_fence16(v0);
+        bool ok = true;
+        if (active) {
+          for (int sub = 0; sub < n_sub; ++sub) {
+            const int it = kit * n_sub + sub, buf = it & 1;
+            if (!(ok = mbar_wait(bar(kPBarS + buf), (it >> 1) & 1, a.status)) || *s_abort) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            // 64 scores in four loads of 16 columns, each in flight while the
+            // previous ones are summed (a wait covers every earlier load; the
+            // fence keeps the compiler from reading a register before it)
+            const uint32_t tS = tmem + 256 * buf + 128 * hl + 64 * qh + lane_base;
+            uint32_t v0[16], v1[16];
+            tmem_ld16(tS, v0);
+            tmem_wait_ld();
+            reg_fence16(v0);
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            uint32_t (&cur)[16] = (c & 1) ? v1 : v0;
-            uint32_t (&nxt)[16] = (c & 1) ? v0 : v1;
-            if (c < 7) {
-              tmem_ld16(tS + 16 * (c + 1), nxt);
-            } else {
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(bar(kPBarFree + g / 2));  // the tile may be refilled
-            }
-            sum16(cur);
-            if (c < 7) {
-              tmem_wait_ld();
-              reg_fence16(nxt);
+            for (int c = 0; c < 4; ++c) {
+              uint32_t (&cur)[16] = (c & 1) ? v1 : v0;
+              uint32_t (&nxt)[16] = (c & 1) ? v0 : v1;
+              if (c < 3) {
+                tmem_ld16(tS + 16 * (c + 1), nxt);
+              } else {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(kPBarFree + buf));  // the buffer may be refilled
+              }
+              sum16(cur);
+              if (c < 3) {
+                tmem_wait_ld();
+                reg_fence16(nxt);
+              }
             }
           }
+        }
+        if (!ok) {
+          *s_abort = 1;
+          break;
         }
         float a0, a1, a2, a3;
         f2_unpack(f2_add(A[0], A[1]), a0, a1);
         f2_unpack(f2_add(A[2], A[3]), a2, a3);
         const float acc = (a0 + a1) + (a2 + a3);
-        // Heads 1-3 hand their sums to head 0's warpgroup through shared memory
+        // Warpgroups 1.. hand their sums to warpgroup 0 through shared memory
         // (slot double-buffered by block parity, guarded by bounded mbarrier
-        // waits).  Head 0's warpgroup adds them one block late, while its own
-        // next block is under way, so it never waits for the slowest head.
-        if (g > 0) {
-          const int sl = it & 1;
-          if (it >= 2 && !mbar_wait(bar(kPBarRedEmpty + sl), ((it >> 1) - 1) & 1, a.status)) { *s_abort = 1; break; }
-          red[(sl * 3 + g - 1) * kTile + key] = acc;
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(kPBarRedFull + sl));
+        // waits).  Warpgroup 0 adds them one block late, while its own next
+        // block is under way, so it never waits for the slowest one.
+        if (w > 0) {
+          if (active) {
+            const int sl = kit & 1;
+            if (kit >= 2 && !mbar_wait(bar(kPBarRedEmpty + sl), ((kit >> 1) - 1) & 1, a.status)) { *s_abort = 1; break; }
+            red[(sl * 3 + w - 1) * kTile + key] = acc;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kPBarRedFull + sl));
+          }
         } else {
-          if (jb > 0 && !combine(rd, it - 1, jb - 1, pend)) break;
+          if (jb > 0 && !combine(rd, kit - 1, jb - 1, pend)) break;
           pend = acc;
         }
       }
-      // head 0's warpgroup: the round's last block
-      if (g == 0 && nblk > 0 && !*s_abort) combine(rd, it0 + nblk - 1, nblk - 1, pend);
+      // warpgroup 0: the round's last block
+      if (w == 0 && nblk > 0 && !*s_abort) combine(rd, kit0 + nblk - 1, nblk - 1, pend);
       __syncthreads();
     }
   }
@@ -832,7 +867,9 @@ static cudaError_t launch_attn(const PrefillParams& p, bool gather, cudaStream_t
   a.scale_log2 = (float)((double)p.scale * 1.4426950408889634);
   a.out = p.out; a.lse = p.lse; a.status = p.status;
   const int ntile = p.G >= 2 ? 2 : 1;
-  dim3 grid(n_tiles, p.Hq / ntile, p.B);
+  const uint64_t n_ctas = (uint64_t)n_tiles * (uint64_t)(p.Hq / ntile) * (uint64_t)p.B;
+  if (n_ctas >= (1ull << 31)) return cudaErrorNotSupported;
+  dim3 grid((unsigned)n_ctas);
   // The kernel's setmaxnreg split assumes exactly kLaunchRegs registers per
   // thread at launch; with fewer, the softmax warpgroups' increase could never
   // be satisfied.  Refuse to launch a build that does not match.
@@ -869,8 +906,9 @@ cudaError_t launch_prefill_anchor(const PrefillParams& p, cudaStream_t st) {
   if (fa.numRegs != kPoolLaunchRegs) return cudaErrorNotSupported;
   e = cudaFuncSetAttribute(pool, cudaFuncAttributeMaxDynamicSharedMemorySize, kPoolSmem);
   if (e != cudaSuccess) return e;
-  dim3 grid(n_tiles - 1, p.Hkv, p.B);
-  pool<<<grid, kPoolThreads, kPoolSmem, st>>>(tq, tk, a);
+  const uint64_t n_pool = (uint64_t)(n_tiles - 1) * (uint64_t)p.Hkv * (uint64_t)p.B;
+  if (n_pool >= (1ull << 31)) return cudaErrorNotSupported;
+  pool<<<dim3((unsigned)n_pool), kPoolThreads, kPoolSmem, st>>>(tq, tk, a);
   return cudaGetLastError();
 }
 
