@@ -51,12 +51,10 @@ def parse():
 
 
 # DRAM bytes per call (dram__bytes_read.sum + dram__bytes_write.sum of the
-# call's kernels) from the ncu capture summarised in the named profile; set an
-# entry to None when one of its kernels changes until it is captured again.
-# (The pooling kernel's exp split between SFU and FMA pipe changed after the
-# capture; that moves no memory traffic.)
+# call's kernels) from the ncu capture summarised in the named profile; None
+# while one of the call's kernels has changed since that capture.
 NCU_TRAFFIC = {
-    "prefill_anchor": {"bytes": (201420800 + 98343424) + (168611072 + 19121664),
+    "prefill_anchor": {"bytes": None,  # the pooling kernel changed (double-buffered S^T)
                        "profile": "profiles/traffic_prefill_n16384_decode_b16_t32768.md"},
     "decode_anchor": {"bytes": 2147660032 + 24662784 + 75661056 + 187648,
                       "profile": "profiles/traffic_prefill_n16384_decode_b16_t32768.md"},
