@@ -269,12 +269,35 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       }
       for (int j = 0; j < nblk; ++j) {
         const int st = j & 1;
+        const bool dense = !GATHER || j == n_gather;
+        // Gathered block: every gather warp loads the block's 128 key indices in
+        // one coalesced round (row 32e + lane in kix[e], its validity in bit lane
+        // of m[e]) before it waits for the stage, so their latency overlaps the
+        // block in flight instead of preceding the copies.
+        int kix[4] = {0, 0, 0, 0};
+        uint32_t m[4] = {0u, 0u, 0u, 0u};
+        if (GATHER && !dense) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int pos = kTile * j + 32 * e + lane;
+            kix[e] = pos < kt ? __ldg(irow + pos) : -1;
+          }
+        }
         prefetch_rows(j + 2);
+        if (GATHER && !dense) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int pos = kTile * j + 32 * e + lane;
+            const bool ok = kix[e] >= 0 && kix[e] < kTile * t;
+            if (gw == 0 && pos < kt && !ok) flag_status(a.status, kStatusBadIndex);
+            m[e] = __ballot_sync(0xffffffffu, ok);
+            if (!ok) kix[e] = kTile * t;  // a valid row; the copy of a masked row is zero-filled
+          }
+        }
         if (j >= 2 && !mbar_wait(bar(kBarKvEmpty + st), ((j >> 1) - 1) & 1, a.status)) { *s_abort = 1; break; }
         if (*s_abort) break;
         const uint32_t kb = sbase + kAttnKV + (2 * st) * kTileBytes;
         const uint32_t vb = kb + kTileBytes;
-        const bool dense = !GATHER || j == n_gather;
         if (dense) {
           if (gw > 0) {
             if (lane == 0) mbar_arrive(bar(kBarKvFull + st));  // helpers complete the count
@@ -287,33 +310,27 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tma_load_2d(vb + kHalfBytes, &tm_v, 64, y, bar(kBarKvFull + st));
           }
         } else {
-          // Gathered block: validity of rows 32e + lane -> ballot word e (bit = row & 31).
-          uint32_t m[4] = {0u, 0u, 0u, 0u};
-          if (gw == 0) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int pos = kTile * j + 32 * e + lane;
-              const int key = pos < kt ? __ldg(irow + pos) : -1;
-              const bool ok = key >= 0 && key < kTile * t;
-              if (pos < kt && !ok) flag_status(a.status, kStatusBadIndex);
-              m[e] = __ballot_sync(0xffffffffu, ok);
-            }
-          }
           // Copy: each warp instruction moves two whole 256-byte rows (16 lanes per
           // row, one 16-byte chunk each) into the swizzled layout; masked rows are
           // zero-filled from a valid address.  The gather warps take every third
-          // pair of rows.
+          // pair of rows; a row's index comes from the lane that loaded it.
           const int c16 = lane & 15;
           const uint32_t half = (uint32_t)(c16 >> 3) * kHalfBytes;
-          for (int s2 = gw; s2 < kTile / 2; s2 += kGatherWarps) {
-            const int row = 2 * s2 + (lane >> 4);
-            const int pos = kTile * j + row;
-            const int key = pos < kt ? __ldg(irow + pos) : -1;
-            const bool ok = key >= 0 && key < kTile * t;
-            const int64_t src = (int64_t)kv_row0 + (ok ? key : kTile * t);
-            const uint32_t off = half + (uint32_t)row * 128u + ((uint32_t)((c16 & 7) ^ (row & 7)) << 4);
-            cp_async16(kb + off, a.k + src * kHeadDim + c16 * 8, ok ? 16u : 0u);
-            cp_async16(vb + off, a.v + src * kHeadDim + c16 * 8, ok ? 16u : 0u);
+#pragma unroll
+          for (int i = 0; i < (kTile / 2 + kGatherWarps - 1) / kGatherWarps; ++i) {
+            const int s2 = gw + kGatherWarps * i;  // warp-uniform
+            if (s2 < kTile / 2) {
+              const int row = 2 * s2 + (lane >> 4);
+              const int e = s2 >> 4;  // = row >> 5 for both rows of the pair
+              const int ke = e == 0 ? kix[0] : e == 1 ? kix[1] : e == 2 ? kix[2] : kix[3];
+              const uint32_t me = e == 0 ? m[0] : e == 1 ? m[1] : e == 2 ? m[2] : m[3];
+              const int key = __shfl_sync(0xffffffffu, ke, row & 31);
+              const bool ok = (me >> (row & 31)) & 1u;
+              const int64_t src = (int64_t)kv_row0 + key;
+              const uint32_t off = half + (uint32_t)row * 128u + ((uint32_t)((c16 & 7) ^ (row & 7)) << 4);
+              cp_async16(kb + off, a.k + src * kHeadDim + c16 * 8, ok ? 16u : 0u);
+              cp_async16(vb + off, a.v + src * kHeadDim + c16 * 8, ok ? 16u : 0u);
+            }
           }
           cp_async_commit();
           cp_async_wait<0>();

@@ -9,7 +9,7 @@ import oracle as O
 from long_context_emitting_b200 import api, workload
 from long_context_emitting_b200.schedule import PrefillSchedule
 from _compare import (assert_attention_close, assert_index_set_ok, assert_pooled_close,
-                      LSE_ABS)
+                      LSE_ABS, O_REL_L2, rel_l2)
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda")
@@ -146,6 +146,50 @@ def test_prefill_n262144_sampled_tiles():
     # a middle and the last query tiles
     cfg = workload.scaled(workload.PREFILL_64K, name="prefill_b1_n262144", N=262144)
     _check(cfg, tiles=[0, 1, 1024, 2047])
+
+
+def test_prefill_growing_scores_rescale_running_max():
+    # Key norms grow along the sequence (x1 at the start to x8 at the end), so a
+    # row's later key blocks exceed its running maximum by more than the 2^8
+    # threshold and the kernel must rescale O and l mid-row; checked against the
+    # oracle on every tile, anchor and reuse.
+    cfg = workload.scaled(workload.PREFILL_16K, name="prefill_growing", N=1024)
+    inp = workload.prefill_layer(cfg, 0, DEV)
+    grow = torch.linspace(1.0, 8.0, cfg.N, device=DEV).view(1, 1, cfg.N, 1)
+    inp["k"] = (inp["k"].float() * grow).to(torch.bfloat16)
+    sch = PrefillSchedule(cfg.B, cfg.Hq, cfg.Hkv, cfg.N, (0,), 2, DEV)
+    out = torch.empty_like(inp["q"])
+    sch.run_anchor(inp, out)
+    lse = sch.lse.clone()
+    sch.run_topk()
+    hm = torch.arange(cfg.Hkv, dtype=torch.int32, device=DEV)
+    out_r = torch.empty_like(out)
+    sch.run_reuse(inp, hm, out_r)  # the same layer reused: its own indices
+    assert api.device_status() == 0
+    q, k, v = (_np(inp[n][0]) for n in ("q", "k", "v"))
+    o_ref, lse_ref, pooled_ref = O.prefill_anchor(q, k, v, SCALE, tile=TILE)
+    # The softmax here is peaked, so |O| reaches ~5, where rounding P and O to bf16
+    # alone is ~2e-2 (a numpy emulation of the kernel's arithmetic -- block-wise
+    # running maximum with the 2^8 threshold, bf16 P, fp32 sums, bf16 O -- gives
+    # 2.0e-2 on this input).  Bound: 2^-8 (max|O| + max|V|), with rel-L2 1e-2.
+    bound = 2.0 ** -8 * (np.abs(o_ref).max() + np.abs(v).max())
+
+    def close(got, ref, what):
+        mx = np.abs(got - ref).max()
+        assert mx <= bound, f"{what}: max-abs {mx:.3e} > {bound:.3e}"
+        assert rel_l2(got, ref) <= O_REL_L2, what
+
+    close(_np(out[0]), o_ref, "anchor O (growing scores)")
+    np.testing.assert_allclose(_np(lse[0]), lse_ref, atol=LSE_ABS, rtol=0)
+    nt = cfg.N // TILE
+    idx = sch.idx[0].cpu().numpy().astype(np.int64)
+    idx_k = np.array([[O.k_for_len(TILE * t)] * cfg.Hkv for t in range(nt)])
+    for t in range(1, nt):
+        for h in range(cfg.Hkv):
+            assert_pooled_close(sch.pooled[0, t, h, :TILE * t].cpu().numpy(), pooled_ref[t, h, :TILE * t],
+                                f"pooled t={t} h={h} (growing scores)")
+    o_r, _ = O.prefill_reuse(q, k, v, idx, idx_k, hm.cpu().numpy(), SCALE, tile=TILE)
+    close(_np(out_r[0]), o_r, "reuse O (growing scores)")
 
 
 def test_prefill_reuse_full_prefix_is_dense():
