@@ -7,11 +7,17 @@
 // 技術的詳細 › アンカーレイヤーと再利用レイヤー and › ヘッドリマッピング.
 //
 // prefill_attn_kernel<GATHER, F16>  (F16: fp16 data, else bf16)
-//   One CTA per (query tile t, pair of query heads of one GQA group, sequence),
-//   launched longest tiles first over the whole grid.
+//   Work item: (query tile t, pair of query heads of one GQA group, sequence);
+//   the grid has one CTA per item, in item order (longest tiles first).  CTAs
+//   are persistent: when a CTA's producer reaches the last key block of its
+//   item it asks the hardware (cluster launch control) to cancel the launch of
+//   the next CTA that has not started and takes over that CTA's item, so
+//   about one CTA per SM runs all items in launch order, and the next item's
+//   query tiles and key blocks load while the current item finishes.
 //   The two heads share every K/V block, so each block is loaded once for two
 //   128 x 128 attention tiles.  Warp roles (384 threads, three warpgroups):
-//     warp 8      TMA producer: Q tiles, then K/V blocks into a 2-stage ring.
+//     warp 8      TMA producer: Q tiles, then K/V blocks into a 2-stage ring
+//                 that continues across the CTA's items; scheduling requests.
 //                 anchor: dense key blocks 0..t (block t is the diagonal);
 //                 reuse: the anchor's indices of row (t, head_map[h]) gathered
 //                 with cp.async (two whole rows per warp instruction) into the
@@ -27,7 +33,8 @@
 //                 rescaled); P goes back to TMEM as bf16 over the row's S, in
 //                 two halves of 64 keys, each handed to the MMA as soon as it
 //                 is stored (PV of the first half overlaps the exponentials of
-//                 the second).
+//                 the second).  Each warp writes its 32 rows of O through a
+//                 swizzled shared-memory stage and TMA stores.
 //   The MMA thread alternates between the tiles, so the tensor cores work on
 //   one tile while the other tile's softmax runs.  The softmax warpgroups take
 //   registers from the third one (setmaxnreg; the launch checks the split).
@@ -80,9 +87,20 @@ static_assert((kLaunchRegs - kOtherRegs) * 128 >= (kSoftmaxRegs - kLaunchRegs) *
 static_assert(kLaunchRegs * kAttnThreads <= 65536, "launch registers exceed the SM");
 constexpr uint32_t kAttnQ = 0;                         // 2 query tiles
 constexpr uint32_t kAttnKV = 2 * kTileBytes;           // stage s: K at +2s*tile, V at +(2s+1)*tile
-constexpr uint32_t kAttnMisc = kAttnKV + 4 * kTileBytes;
-constexpr uint32_t kAttnSmem = kAttnMisc + 256 + 1024;  // misc + alignment slack
-enum { kBarQ = 0, kBarKvFull = 1, kBarKvEmpty = 3, kBarS = 5, kBarP = 7, kBarO = 11, kAttnBars = 13 };
+// O staging for the TMA stores: per softmax warp 32 rows x 64 columns (4 KB)
+constexpr uint32_t kAttnStage = kAttnKV + 4 * kTileBytes;
+constexpr uint32_t kStageWarpBytes = 32u * 128u;
+constexpr uint32_t kAttnMisc = kAttnStage + 8 * kStageWarpBytes;
+// misc: barriers, TMEM address, abort flag, gather masks, scheduling responses
+constexpr uint32_t kMiscTmem = 192, kMiscAbort = 200, kMiscMasks = 224, kMiscClc = 256, kMiscItem = 288;
+constexpr uint32_t kAttnSmem = kAttnMisc + 512 + 1024;  // misc + alignment slack
+static_assert(kAttnSmem <= 227u * 1024u, "attention shared memory exceeds the per-block limit");
+// QFree: the item's S MMAs have read its query tiles; ClcFull: a scheduling
+// response has landed (read by the producer); Item: the producer has
+// published the next item in its slot; ClcEmpty: every other role has read it
+enum { kBarQ = 0, kBarKvFull = 1, kBarKvEmpty = 3, kBarS = 5, kBarP = 7, kBarO = 11, kBarQFree = 13,
+       kBarClcFull = 14, kBarClcEmpty = 16, kBarItem = 18, kAttnBars = 20 };
+static_assert(kAttnBars * 8 <= kMiscTmem, "attention barriers overlap the misc fields");
 
 // ---- pooling kernel layout ----
 constexpr int kPoolThreads = 640;  // warpgroup 0: TMA (warp 0), MMA (warp 1), TMEM owner (warp 2);
@@ -155,67 +173,141 @@ __device__ __forceinline__ constexpr uint64_t qpair_step(int ks) {
   return (uint64_t)(((uint32_t)(ks >> 2) * 4u * kHalfBytes + (uint32_t)(ks & 3) * 32u) >> 4);
 }
 
+// One unit of work of the attention kernel: query tile t of heads g0 .. g0 +
+// ntile - 1 (one GQA group, key head h) of sequence b, with its key blocks.
+// Item order (the grid's, kept by taking over pending CTAs in launch order):
+// anchor: longest tiles first over the whole grid (every head group and
+// sequence of tile t before any of tile t - 1), so no long tile starts late;
+// reuse: tiles longest first within each head group, the head groups one
+// after another (the CTAs running together then gather from the same key
+// head's rows, which measured faster than the global order).
+struct AttnItem {
+  int t, g0, b, h;
+  int nblk;      // key blocks: anchor 0..t; reuse n_gather gathered + the diagonal
+  int n_gather;  // reuse: gathered blocks (kt keys of the anchor's row)
+  int kt;
+  const int32_t* irow;
+  int64_t q_row0;
+  int kv_row0;
+};
+
+// The item's fields from its index and (reuse) the two values read from
+// device memory: kt keys in the anchor's index row and the anchor key head am
+// (already checked; kt = 0 when the row was unusable).
+template <bool GATHER>
+__device__ __forceinline__ AttnItem attn_item_of(const AttnArgs& a, int item, int ntile, int kt, int am) {
+  AttnItem w;
+  const int HG = a.Hq / ntile;
+  int rem;
+  if (GATHER) {
+    w.t = a.n_tiles - 1 - item % a.n_tiles;
+    rem = item / a.n_tiles;
+  } else {
+    w.t = a.n_tiles - 1 - item / (HG * a.B);
+    rem = item % (HG * a.B);
+  }
+  w.g0 = (rem % HG) * ntile;
+  w.b = rem / HG;
+  w.h = w.g0 / a.G;
+  w.kt = GATHER ? kt : 0;
+  w.irow = GATHER ? a.idx + (((int64_t)w.b * a.n_tiles + w.t) * a.Hkv + am) * a.k_max : nullptr;
+  w.n_gather = (w.kt + kTile - 1) / kTile;
+  w.nblk = GATHER ? w.n_gather + 1 : w.t + 1;
+  w.q_row0 = ((int64_t)w.b * a.Hq + w.g0) * a.N + (int64_t)kTile * w.t;
+  w.kv_row0 = (int)(((int64_t)w.b * a.Hkv + w.h) * a.N);
+  return w;
+}
+
+// Reads (reuse) the item's anchor head and index count and checks them;
+// returns kt and am for attn_item_of.
+template <bool GATHER>
+__device__ __forceinline__ void attn_item_load(const AttnArgs& a, int item, int ntile, bool flag_errors,
+                                               int& kt, int& am) {
+  kt = 0;
+  am = 0;
+  if (GATHER) {
+    const int HG = a.Hq / ntile;
+    const int t = a.n_tiles - 1 - item % a.n_tiles;
+    const int rem = item / a.n_tiles;
+    const int b = rem / HG, h = (rem % HG) * ntile / a.G;
+    const int m = a.head_map[h];
+    bool ok = m >= 0 && m < a.Hkv;
+    if (ok) {
+      const int64_t row = ((int64_t)b * a.n_tiles + t) * a.Hkv + m;
+      kt = a.idx_k[row];
+      ok = kt >= 0 && kt <= a.k_max && kt <= kTile * t;
+      am = m;
+    }
+    if (!ok) {
+      if (flag_errors) flag_status(a.status, kStatusBadIndex);
+      kt = 0;
+      am = 0;
+    }
+  }
+}
+
+template <bool GATHER>
+__device__ __forceinline__ AttnItem attn_item(const AttnArgs& a, int item, int ntile, bool flag_errors) {
+  int kt, am;
+  attn_item_load<GATHER>(a, item, ntile, flag_errors, kt, am);
+  return attn_item_of<GATHER>(a, item, ntile, kt, am);
+}
+
 template <bool GATHER, bool F16>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                    const AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   uint8_t* misc = smem + kAttnMisc;
   uint64_t* bars = reinterpret_cast<uint64_t*>(misc);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 128);
-  volatile int* s_abort = reinterpret_cast<volatile int*>(misc + 136);
-  uint32_t* masks = reinterpret_cast<uint32_t*>(misc + 160);        // [2 stages][4]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + kMiscTmem);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(misc + kMiscAbort);
+  uint32_t* masks = reinterpret_cast<uint32_t*>(misc + kMiscMasks);  // [2 stages][4]
+  const uint32_t clc_resp = smem_u32(misc + kMiscClc);                // [2] x 16 bytes
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // 1-D grid.  Anchor: longest tiles first over the whole grid (every head
-  // group and sequence of tile t before any of tile t - 1), so no long tile
-  // starts late.  Reuse: tiles longest first within each head group, the head
-  // groups one after another (the CTAs running together then gather from the
-  // same key head's rows, which measured faster than the global order).
   const int ntile = a.G >= 2 ? 2 : 1;
-  const int HG = a.Hq / ntile;
-  int t, rem;
-  if (GATHER) {
-    t = a.n_tiles - 1 - (int)(blockIdx.x % a.n_tiles);
-    rem = (int)(blockIdx.x / a.n_tiles);
-  } else {
-    t = a.n_tiles - 1 - (int)(blockIdx.x / (HG * a.B));
-    rem = (int)(blockIdx.x % (HG * a.B));
-  }
-  const int g0 = (rem % HG) * ntile;
-  const int b = rem / HG;
-  const int h = g0 / a.G;
-
-  // ---- key blocks ------------------------------------------------------------
-  int n_gather = 0, kt = 0;
-  const int32_t* irow = nullptr;
-  if (GATHER) {
-    const int am = a.head_map[h];
-    bool ok = am >= 0 && am < a.Hkv;
-    if (ok) {
-      const int64_t row = ((int64_t)b * a.n_tiles + t) * a.Hkv + am;
-      kt = a.idx_k[row];
-      irow = a.idx + row * a.k_max;
-      ok = kt >= 0 && kt <= a.k_max && kt <= kTile * t;
+  // Persistent CTAs: a CTA starts with item blockIdx.x; while working on its
+  // item at position pos of its sequence it asks (request pos) to take over
+  // the next CTA of the grid that has not started, and continues with that
+  // CTA's item.  The K/V stage ring and the per-block barriers run on one
+  // block counter g over all the CTA's items, so the next item's loads and
+  // its first S MMAs overlap the current item's last blocks and epilogue.
+  // The producer asks for the next item when it reaches the current item's
+  // last key block (late enough that the item taken is the next one due, early
+  // enough that its loads start before this item's compute ends), reads the
+  // item's anchor head and index count, and publishes {item, kt, am} in slot
+  // pos & 1 of shared memory.  Readers of a slot besides the producer warp:
+  // the MMA warp, the softmax warps in use and (reuse) the two gather helpers.
+  int* item_slot = reinterpret_cast<int*>(misc + kMiscItem);  // [2][4]
+  const uint32_t n_clc_readers = 1u + 4u * (uint32_t)ntile + (GATHER ? 2u : 0u);
+  auto read_item = [&](int pos, int& kt, int& am) -> int {  // one thread
+    int nx = -1;
+    kt = 0;
+    am = 0;
+    if (mbar_wait(bar(kBarItem + (pos & 1)), (pos >> 1) & 1, a.status)) {
+      const volatile int* sl = item_slot + 4 * (pos & 1);
+      nx = sl[0];
+      kt = sl[1];
+      am = sl[2];
+    } else {
+      *s_abort = 1;
     }
-    if (!ok) {
-      if (tid == 0) flag_status(a.status, kStatusBadIndex);
-      kt = 0;
-    }
-    n_gather = (kt + kTile - 1) / kTile;
-  }
-  const int nblk = GATHER ? n_gather + 1 : t + 1;
-  const int64_t q_row0 = ((int64_t)b * a.Hq + g0) * a.N + (int64_t)kTile * t;
-  const int kv_row0 = (int)(((int64_t)b * a.Hkv + h) * a.N);
+    mbar_arrive(bar(kBarClcEmpty + (pos & 1)));
+    return nx;
+  };
 
   if (tid == 0) {
     for (int i = 0; i < kAttnBars; ++i) {
-      const bool per_warp = i >= kBarP && i < kBarP + 4;  // 4 softmax warps per tile
-      const bool kv_full = i >= kBarKvFull && i < kBarKvFull + 2;  // reuse: one arrival per gather warp
-      mbar_init(bar(i), per_warp ? 4u : (kv_full && GATHER ? (uint32_t)kGatherWarps : 1u));
+      uint32_t count = 1;
+      if (i >= kBarP && i < kBarP + 4) count = 4;  // 4 softmax warps per tile
+      if (GATHER && i >= kBarKvFull && i < kBarKvFull + 2) count = kGatherWarps;  // one arrival per gather warp
+      if (i >= kBarClcEmpty && i < kBarClcEmpty + 2) count = n_clc_readers;  // (Item: the producer, 1)
+      mbar_init(bar(i), count);
     }
     *s_abort = 0;
     mbar_fence_init();
@@ -235,27 +327,20 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int gw = warp == kProducerWarp ? 0 : (warp >= 10 ? warp - 9 : -1);
     if (gw == 0 || (GATHER && gw > 0)) {
       // ================================ TMA producer ================================
-      if (gw == 0 && lane == 0) {
-        mbar_expect_tx(bar(kBarQ), ntile * kTileBytes);
-        for (int i = 0; i < ntile; ++i) {
-          const int y = (int)(q_row0 + (int64_t)i * a.N);
-          tma_load_2d(sbase + kAttnQ + i * kTileBytes, &tm_q, 0, y, bar(kBarQ));
-          tma_load_2d(sbase + kAttnQ + i * kTileBytes + kHalfBytes, &tm_q, 64, y, bar(kBarQ));
-        }
-      }
+      const bool leader = gw == 0 && lane == 0;  // issues TMA copies and the scheduling requests
       // Reuse: the gathered rows of a layer are first read from DRAM at scattered
       // positions; their latency would exceed a block's compute.  Each gather warp
       // pulls its share of the rows of block j + 2 into L2 before it waits for
       // the stage of block j, so the later copies are L2 hits.
-      auto prefetch_rows = [&](int jp) {
+      auto prefetch_rows = [&](const AttnItem& w, int jp) {
         if constexpr (GATHER) {
-          if (jp >= n_gather) return;
+          if (jp >= w.n_gather) return;
           for (int r = gw + kGatherWarps * lane; r < kTile; r += kGatherWarps * 32) {
             const int pos = kTile * jp + r;
-            if (pos >= kt) break;
-            const int key = __ldg(irow + pos);
-            if (key < 0 || key >= kTile * t) continue;  // flagged when the block is gathered
-            const int64_t off = ((int64_t)kv_row0 + key) * kHeadDim;
+            if (pos >= w.kt) break;
+            const int key = __ldg(w.irow + pos);
+            if (key < 0 || key >= kTile * w.t) continue;  // flagged when the block is gathered
+            const int64_t off = ((int64_t)w.kv_row0 + key) * kHeadDim;
             prefetch_l2(a.k + off);
             prefetch_l2(a.k + off + 64);
             prefetch_l2(a.v + off);
@@ -263,88 +348,166 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           }
         }
       };
-      if (GATHER) {
-        prefetch_rows(0);
-        prefetch_rows(1);
-      }
-      for (int j = 0; j < nblk; ++j) {
-        const int st = j & 1;
-        const bool dense = !GATHER || j == n_gather;
-        // Gathered block: every gather warp loads the block's 128 key indices in
-        // one coalesced round (row 32e + lane in kix[e], its validity in bit lane
-        // of m[e]) before it waits for the stage, so their latency overlaps the
-        // block in flight instead of preceding the copies.
-        int kix[4] = {0, 0, 0, 0};
-        uint32_t m[4] = {0u, 0u, 0u, 0u};
-        if (GATHER && !dense) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int pos = kTile * j + 32 * e + lane;
-            kix[e] = pos < kt ? __ldg(irow + pos) : -1;
-          }
+      // The item's query tiles (leader).  Their buffer is free once the previous
+      // item's S MMAs have read it.
+      auto load_q = [&](const AttnItem& w) {
+        mbar_expect_tx(bar(kBarQ), ntile * kTileBytes);
+        for (int i = 0; i < ntile; ++i) {
+          const int y = (int)(w.q_row0 + (int64_t)i * a.N);
+          tma_load_2d(sbase + kAttnQ + i * kTileBytes, &tm_q, 0, y, bar(kBarQ));
+          tma_load_2d(sbase + kAttnQ + i * kTileBytes + kHalfBytes, &tm_q, 64, y, bar(kBarQ));
         }
-        prefetch_rows(j + 2);
-        if (GATHER && !dense) {
+      };
+      AttnItem it = attn_item<GATHER>(a, blockIdx.x, ntile, leader);
+      prefetch_rows(it, 0);
+      prefetch_rows(it, 1);
+      uint32_t g = 0;            // key blocks of the CTA's earlier items
+      int unread = -1;           // leader: a request whose response it has not read
+      if (leader) load_q(it);  // later items' tiles are loaded as the previous item ends
+      for (int pos = 0;; ++pos) {
+        bool ok = !__any_sync(0xffffffffu, *s_abort != 0);
+        for (int j = 0; ok && j < it.nblk; ++j) {
+          const uint32_t gb = g + (uint32_t)j;
+          const int st = (int)(gb & 1u);
+          const bool dense = !GATHER || j == it.n_gather;
+          // Gathered block: every gather warp loads the block's 128 key indices in
+          // one coalesced round (row 32e + lane in kix[e], its validity in bit lane
+          // of m[e]) before it waits for the stage, so their latency overlaps the
+          // block in flight instead of preceding the copies.
+          int kix[4] = {0, 0, 0, 0};
+          uint32_t m[4] = {0u, 0u, 0u, 0u};
+          if (GATHER && !dense) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int pos = kTile * j + 32 * e + lane;
-            const bool ok = kix[e] >= 0 && kix[e] < kTile * t;
-            if (gw == 0 && pos < kt && !ok) flag_status(a.status, kStatusBadIndex);
-            m[e] = __ballot_sync(0xffffffffu, ok);
-            if (!ok) kix[e] = kTile * t;  // a valid row; the copy of a masked row is zero-filled
-          }
-        }
-        if (j >= 2 && !mbar_wait(bar(kBarKvEmpty + st), ((j >> 1) - 1) & 1, a.status)) { *s_abort = 1; break; }
-        if (*s_abort) break;
-        const uint32_t kb = sbase + kAttnKV + (2 * st) * kTileBytes;
-        const uint32_t vb = kb + kTileBytes;
-        if (dense) {
-          if (gw > 0) {
-            if (lane == 0) mbar_arrive(bar(kBarKvFull + st));  // helpers complete the count
-          } else if (lane == 0) {
-            mbar_expect_tx(bar(kBarKvFull + st), 2 * kTileBytes);
-            const int y = kv_row0 + kTile * (GATHER ? t : j);
-            tma_load_2d(kb, &tm_k, 0, y, bar(kBarKvFull + st));
-            tma_load_2d(kb + kHalfBytes, &tm_k, 64, y, bar(kBarKvFull + st));
-            tma_load_2d(vb, &tm_v, 0, y, bar(kBarKvFull + st));
-            tma_load_2d(vb + kHalfBytes, &tm_v, 64, y, bar(kBarKvFull + st));
-          }
-        } else {
-          // Copy: each warp instruction moves two whole 256-byte rows (16 lanes per
-          // row, one 16-byte chunk each) into the swizzled layout; masked rows are
-          // zero-filled from a valid address.  The gather warps take every third
-          // pair of rows; a row's index comes from the lane that loaded it.
-          const int c16 = lane & 15;
-          const uint32_t half = (uint32_t)(c16 >> 3) * kHalfBytes;
-#pragma unroll
-          for (int i = 0; i < (kTile / 2 + kGatherWarps - 1) / kGatherWarps; ++i) {
-            const int s2 = gw + kGatherWarps * i;  // warp-uniform
-            if (s2 < kTile / 2) {
-              const int row = 2 * s2 + (lane >> 4);
-              const int e = s2 >> 4;  // = row >> 5 for both rows of the pair
-              const int ke = e == 0 ? kix[0] : e == 1 ? kix[1] : e == 2 ? kix[2] : kix[3];
-              const uint32_t me = e == 0 ? m[0] : e == 1 ? m[1] : e == 2 ? m[2] : m[3];
-              const int key = __shfl_sync(0xffffffffu, ke, row & 31);
-              const bool ok = (me >> (row & 31)) & 1u;
-              const int64_t src = (int64_t)kv_row0 + key;
-              const uint32_t off = half + (uint32_t)row * 128u + ((uint32_t)((c16 & 7) ^ (row & 7)) << 4);
-              cp_async16(kb + off, a.k + src * kHeadDim + c16 * 8, ok ? 16u : 0u);
-              cp_async16(vb + off, a.v + src * kHeadDim + c16 * 8, ok ? 16u : 0u);
+            for (int e = 0; e < 4; ++e) {
+              const int pos_k = kTile * j + 32 * e + lane;
+              kix[e] = pos_k < it.kt ? __ldg(it.irow + pos_k) : -1;
             }
           }
-          cp_async_commit();
-          cp_async_wait<0>();
-          fence_proxy_async_smem();  // the tensor cores read these rows through the async proxy
-          __syncwarp();
-          if (lane == 0) {
-            if (gw == 0) {
-#pragma unroll
-              for (int e = 0; e < 4; ++e) masks[st * 4 + e] = m[e];
+          prefetch_rows(it, j + 2);
+          if (leader && j == it.nblk - 1) {
+            // request the item after this one (slot pos & 1, free once every
+            // reader has taken item pos - 1 from it)
+            if (pos < 2 || mbar_wait(bar(kBarClcEmpty + (pos & 1)), ((pos >> 1) - 1) & 1, a.status)) {
+              mbar_expect_tx(bar(kBarClcFull + (pos & 1)), 16);
+              clc_try_cancel(clc_resp + 16u * (uint32_t)(pos & 1), bar(kBarClcFull + (pos & 1)));
+              unread = pos;
+            } else {
+              *s_abort = 1;
             }
-            mbar_arrive(bar(kBarKvFull + st));  // release: rows (and masks) visible
+          }
+          if (GATHER && !dense) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int pos_k = kTile * j + 32 * e + lane;
+              const bool v = kix[e] >= 0 && kix[e] < kTile * it.t;
+              if (gw == 0 && pos_k < it.kt && !v) flag_status(a.status, kStatusBadIndex);
+              m[e] = __ballot_sync(0xffffffffu, v);
+              if (!v) kix[e] = kTile * it.t;  // a valid row; the copy of a masked row is zero-filled
+            }
+          }
+          if (gb >= 2 && !mbar_wait(bar(kBarKvEmpty + st), ((gb >> 1) - 1) & 1, a.status)) *s_abort = 1;
+          if (__any_sync(0xffffffffu, *s_abort != 0)) {
+            ok = false;
+            break;
+          }
+          const uint32_t kb = sbase + kAttnKV + (2 * st) * kTileBytes;
+          const uint32_t vb = kb + kTileBytes;
+          if (dense) {
+            if (gw > 0) {
+              if (lane == 0) mbar_arrive(bar(kBarKvFull + st));  // helpers complete the count
+            } else if (lane == 0) {
+              mbar_expect_tx(bar(kBarKvFull + st), 2 * kTileBytes);
+              const int y = it.kv_row0 + kTile * (GATHER ? it.t : j);
+              tma_load_2d(kb, &tm_k, 0, y, bar(kBarKvFull + st));
+              tma_load_2d(kb + kHalfBytes, &tm_k, 64, y, bar(kBarKvFull + st));
+              tma_load_2d(vb, &tm_v, 0, y, bar(kBarKvFull + st));
+              tma_load_2d(vb + kHalfBytes, &tm_v, 64, y, bar(kBarKvFull + st));
+            }
+          } else {
+            // Copy: each warp instruction moves two whole 256-byte rows (16 lanes per
+            // row, one 16-byte chunk each) into the swizzled layout; masked rows are
+            // zero-filled from a valid address.  The gather warps take every third
+            // pair of rows; a row's index comes from the lane that loaded it.
+            const int c16 = lane & 15;
+            const uint32_t half = (uint32_t)(c16 >> 3) * kHalfBytes;
+#pragma unroll
+            for (int i = 0; i < (kTile / 2 + kGatherWarps - 1) / kGatherWarps; ++i) {
+              const int s2 = gw + kGatherWarps * i;  // warp-uniform
+              if (s2 < kTile / 2) {
+                const int row = 2 * s2 + (lane >> 4);
+                const int e = s2 >> 4;  // = row >> 5 for both rows of the pair
+                const int ke = e == 0 ? kix[0] : e == 1 ? kix[1] : e == 2 ? kix[2] : kix[3];
+                const uint32_t me = e == 0 ? m[0] : e == 1 ? m[1] : e == 2 ? m[2] : m[3];
+                const int key = __shfl_sync(0xffffffffu, ke, row & 31);
+                const bool v = (me >> (row & 31)) & 1u;
+                const int64_t src = (int64_t)it.kv_row0 + key;
+                const uint32_t off = half + (uint32_t)row * 128u + ((uint32_t)((c16 & 7) ^ (row & 7)) << 4);
+                cp_async16(kb + off, a.k + src * kHeadDim + c16 * 8, v ? 16u : 0u);
+                cp_async16(vb + off, a.v + src * kHeadDim + c16 * 8, v ? 16u : 0u);
+              }
+            }
+            cp_async_commit();
+            cp_async_wait<0>();
+            fence_proxy_async_smem();  // the tensor cores read these rows through the async proxy
+            __syncwarp();
+            if (lane == 0) {
+              if (gw == 0) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) masks[st * 4 + e] = m[e];
+              }
+              mbar_arrive(bar(kBarKvFull + st));  // release: rows (and masks) visible
+            }
           }
         }
+        if (!ok) break;
+        g += (uint32_t)it.nblk;
+        // the next item: the leader reads the response, the item's index row
+        // and publishes it; the helpers take it from the slot
+        int nx = -1, nkt = 0, nam = 0;
+        if (leader) {
+          if (mbar_wait(bar(kBarClcFull + (pos & 1)), (pos >> 1) & 1, a.status)) {
+            nx = clc_response_x(clc_resp + 16u * (uint32_t)(pos & 1));
+            fence_proxy_async_smem();  // read before the slot is written again by the async unit
+            if (nx >= (int)gridDim.x) {  // not a CTA of this grid: stop rather than index with it
+              flag_status(a.status, kStatusBadIndex);
+              *s_abort = 1;
+              nx = -1;
+            }
+          } else {
+            *s_abort = 1;
+          }
+          unread = -1;
+          if (nx >= 0) attn_item_load<GATHER>(a, nx, ntile, true, nkt, nam);
+          int* sl = item_slot + 4 * (pos & 1);
+          sl[0] = nx;
+          sl[1] = nkt;
+          sl[2] = nam;
+          mbar_arrive(bar(kBarItem + (pos & 1)));  // release: the slot's fields
+        } else if (gw > 0 && lane == 0) {
+          nx = read_item(pos, nkt, nam);
+        }
+        nx = __shfl_sync(0xffffffffu, nx, 0);
+        nkt = __shfl_sync(0xffffffffu, nkt, 0);
+        nam = __shfl_sync(0xffffffffu, nam, 0);
+        if (nx < 0 || __any_sync(0xffffffffu, *s_abort != 0)) break;
+        it = attn_item_of<GATHER>(a, nx, ntile, nkt, nam);
+        if (leader) {
+          // its query tiles: toward L2 at once, into shared memory as soon as
+          // this item's last S MMAs have completed
+          for (int i = 0; i < ntile; ++i) {
+            const int y = (int)(it.q_row0 + (int64_t)i * a.N);
+            tma_prefetch_l2_2d(&tm_q, 0, y);
+            tma_prefetch_l2_2d(&tm_q, 64, y);
+          }
+          if (mbar_wait(bar(kBarQFree), pos & 1, a.status)) load_q(it);
+          else *s_abort = 1;
+        }
+        if (__any_sync(0xffffffffu, *s_abort != 0)) break;
+        prefetch_rows(it, 0);
+        prefetch_rows(it, 1);
       }
+      // never leave with a response still to land in shared memory
+      if (leader && unread >= 0) mbar_wait(bar(kBarClcFull + (unread & 1)), (unread >> 1) & 1, a.status);
     } else if (warp == kMmaWarp) {
       // ================================ MMA issuer ==================================
       if (lane == 0) {
@@ -365,6 +528,8 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             umma_ss(d, dq + kmajor_step(k16), dk + kmajor_step(k16), idesc_s, k16 > 0 ? 1u : 0u);
         };
         // P (128 keys as bf16 pairs) sits in columns 0..63 of the tile's S region.
+        // The first PV of an item overwrites O: the softmax warps arrive on P
+        // only after the previous item's epilogue has read O out of TMEM.
         auto issue_pv = [&](int i, int st, bool acc, int k0) {  // keys 16*k0 .. 16*k0+63
           const uint64_t dv = st ? dv1 : dv0;
           const uint32_t d = tmem + 256 * i + 128, pa = tmem + 256 * i;
@@ -372,48 +537,63 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           for (int k16 = k0; k16 < k0 + 4; ++k16)
             umma_ts(d, pa + 8 * k16, dv + mnmajor_step(k16), idesc_o, (acc || k16 > 0) ? 1u : 0u);
         };
-        bool ok = mbar_wait(bar(kBarQ), 0, a.status);
-        for (int j = 0; ok && j < nblk; ++j) {
-          const int st = j & 1;
-          if (!(ok = mbar_wait(bar(kBarKvFull + st), (j >> 1) & 1, a.status))) break;
-          tc_fence_after();
-          if (j == 0) {
-            for (int i = 0; i < ntile; ++i) {
-              issue_s(i, st);
-              umma_commit(bar(kBarS + i));
+        int item = blockIdx.x, kt, am;
+        attn_item_load<GATHER>(a, item, ntile, false, kt, am);
+        uint32_t g = 0;
+        for (int pos = 0;; ++pos) {
+          const int nblk = attn_item_of<GATHER>(a, item, ntile, kt, am).nblk;
+          bool ok = mbar_wait(bar(kBarQ), pos & 1, a.status);
+          for (int j = 0; ok && j < nblk; ++j) {
+            const uint32_t gb = g + (uint32_t)j;
+            const int st = (int)(gb & 1u);
+            const uint32_t ph = gb & 1u;
+            if (!(ok = mbar_wait(bar(kBarKvFull + st), (gb >> 1) & 1, a.status))) break;
+            tc_fence_after();
+            if (j == 0) {
+              for (int i = 0; i < ntile; ++i) {
+                issue_s(i, st);
+                umma_commit(bar(kBarS + i));
+              }
+              if (nblk == 1) umma_commit(bar(kBarQFree));  // the item's last reads of Q
             }
-          }
-          const bool more = j + 1 < nblk;
-          // tile 0: PV of this block, then S of the next block
-          if (!(ok = mbar_spin(bar(kBarP + 0), j & 1, a.status))) break;
-          tc_fence_after();
-          issue_pv(0, st, j > 0, 0);
-          if (!(ok = mbar_spin(bar(kBarP + 1), j & 1, a.status))) break;
-          tc_fence_after();
-          issue_pv(0, st, j > 0, 4);
-          if (more) {
-            if (!(ok = mbar_wait(bar(kBarKvFull + (st ^ 1)), ((j + 1) >> 1) & 1, a.status))) break;
+            const bool more = j + 1 < nblk;
+            // tile 0: PV of this block, then S of the next block
+            if (!(ok = mbar_spin(bar(kBarP + 0), ph, a.status))) break;
             tc_fence_after();
-            issue_s(0, st ^ 1);
-            umma_commit(bar(kBarS + 0));
-          }
-          if (ntile == 2) {
-            if (!(ok = mbar_spin(bar(kBarP + 2), j & 1, a.status))) break;
+            issue_pv(0, st, j > 0, 0);
+            if (!(ok = mbar_spin(bar(kBarP + 1), ph, a.status))) break;
             tc_fence_after();
-            issue_pv(1, st, j > 0, 0);
-            if (!(ok = mbar_spin(bar(kBarP + 3), j & 1, a.status))) break;
-            tc_fence_after();
-            issue_pv(1, st, j > 0, 4);
+            issue_pv(0, st, j > 0, 4);
+            if (more) {
+              if (!(ok = mbar_wait(bar(kBarKvFull + (st ^ 1)), ((gb + 1) >> 1) & 1, a.status))) break;
+              tc_fence_after();
+              issue_s(0, st ^ 1);
+              umma_commit(bar(kBarS + 0));
+              if (ntile == 1 && j + 2 == nblk) umma_commit(bar(kBarQFree));
+            }
+            if (ntile == 2) {
+              if (!(ok = mbar_spin(bar(kBarP + 2), ph, a.status))) break;
+              tc_fence_after();
+              issue_pv(1, st, j > 0, 0);
+              if (!(ok = mbar_spin(bar(kBarP + 3), ph, a.status))) break;
+              tc_fence_after();
+              issue_pv(1, st, j > 0, 4);
+            }
+            umma_commit(bar(kBarKvEmpty + st));  // K/V stage free once these MMAs complete
+            if (ntile == 2 && more) {
+              issue_s(1, st ^ 1);
+              umma_commit(bar(kBarS + 1));
+              if (j + 2 == nblk) umma_commit(bar(kBarQFree));
+            }
+            if (*s_abort) { ok = false; break; }
           }
-          umma_commit(bar(kBarKvEmpty + st));  // K/V stage free once these MMAs complete
-          if (ntile == 2 && more) {
-            issue_s(1, st ^ 1);
-            umma_commit(bar(kBarS + 1));
-          }
-          if (*s_abort) { ok = false; break; }
+          if (!ok) *s_abort = 1;
+          for (int i = 0; i < ntile; ++i) umma_commit(bar(kBarO + i));
+          if (!ok) break;
+          g += (uint32_t)nblk;
+          item = read_item(pos, kt, am);
+          if (item < 0 || *s_abort) break;
         }
-        if (!ok) *s_abort = 1;
-        for (int i = 0; i < ntile; ++i) umma_commit(bar(kBarO + i));
       }
     }
   } else {
@@ -426,133 +606,178 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       const uint32_t tS = tmem + 256 * i + ((uint32_t)((warp & 3) * 32) << 16);  // S (and P)
       const uint32_t tO = tS + 128;
       const float sc = a.scale_log2;  // > 0, so max(s) * sc = max(s * sc)
-      float m_used = -INFINITY, l_sum = 0.f;
-      bool ok = true;
-      for (int j = 0; j < nblk; ++j) {
-        if (!(ok = mbar_wait(bar(kBarS + i), j & 1, a.status)) || *s_abort) { ok = false; break; }
-        tc_fence_after();
-        const bool diag = GATHER ? (j == n_gather) : (j == t);
-        uint32_t mk[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
-        if (GATHER && !diag) {
-          // masks of the gathered rows (written before the stage's full barrier completed)
-          if (!(ok = mbar_wait(bar(kBarKvFull + (j & 1)), (j >> 1) & 1, a.status))) break;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) mk[e] = masks[(j & 1) * 4 + e];
+      int item = blockIdx.x, kt, am;
+      attn_item_load<GATHER>(a, item, ntile, false, kt, am);
+      uint32_t g = 0;
+      for (int pos = 0;; ++pos) {
+        // only the block count and the diagonal block's position stay live
+        // through the block loop (the loop is register-bound)
+        int nblk, jdiag;
+        {
+          const AttnItem it = attn_item_of<GATHER>(a, item, ntile, kt, am);
+          nblk = it.nblk;
+          jdiag = GATHER ? it.n_gather : it.t;
         }
-        if (diag) {
-          // causal diagonal block: key col is visible to row r if col <= r
+        float m_used = -INFINITY, l_sum = 0.f;
+        bool ok = true;
+        for (int j = 0; j < nblk; ++j) {
+          const uint32_t gb = g + (uint32_t)j;
+          if (!(ok = mbar_wait(bar(kBarS + i), gb & 1u, a.status)) || *s_abort) { ok = false; break; }
+          tc_fence_after();
+          const bool diag = j == jdiag;
+          uint32_t mk[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
+          if (GATHER && !diag) {
+            // masks of the gathered rows (written before the stage's full barrier completed)
+            if (!(ok = mbar_wait(bar(kBarKvFull + (gb & 1u)), (gb >> 1) & 1, a.status))) break;
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const int n = r - 32 * c + 1;  // visible keys of this chunk
-            mk[c] = n >= 32 ? 0xffffffffu : (n <= 0 ? 0u : (1u << n) - 1u);
+            for (int e = 0; e < 4; ++e) mk[e] = masks[(gb & 1u) * 4 + e];
           }
-        }
-        uint32_t v[4][32];
+          if (diag) {
+            // causal diagonal block: key col is visible to row r if col <= r
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, v[c]);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 4; ++c) reg_fence32(v[c]);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          if (mk[c] != 0xffffffffu) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (!((mk[c] >> e) & 1u)) v[c][e] = __float_as_uint(-INFINITY);
+            for (int c = 0; c < 4; ++c) {
+              const int n = r - 32 * c + 1;  // visible keys of this chunk
+              mk[c] = n >= 32 ? 0xffffffffu : (n <= 0 ? 0u : (1u << n) - 1u);
+            }
           }
-        }
-        // ---- row maximum of the raw scores
-        float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          uint32_t v[4][32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int e2 = 0; e2 < 16; ++e2)
-            mp[e2 & 3] = fmax3(mp[e2 & 3], __uint_as_float(v[c][2 * e2]), __uint_as_float(v[c][2 * e2 + 1]));
-        const float mr = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
-        const float mloc = mr == -INFINITY ? -INFINITY : mr * sc;
-        float alpha = 1.f;
-        bool rescale = false;
-        if (m_used == -INFINITY) {
-          m_used = mloc;  // first visible key of the row: O and l are still zero
-        } else if (mloc > m_used + kRescaleLog2) {
-          alpha = fast_exp2(m_used - mloc);
-          m_used = mloc;
-          rescale = true;
-        }
-        if (__any_sync(0xffffffffu, rescale)) {
-          // the previous PV of this tile completed before S of this block was committed
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tO + 32 * c, o);
-            tmem_wait_ld();
-            reg_fence32(o);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(tO + 32 * c, o);
-          }
-        }
-        l_sum *= alpha;
-        const float base = (m_used == -INFINITY) ? 0.f : m_used;
-        // ---- p = exp2(s*sc - base), two scores per packed f32x2 FMA; P goes
-        // back as bf16 pairs into columns 0..63 of the row's S (all read).
-        uint64_t L[4] = {0ull, 0ull, 0ull, 0ull};
-        const uint64_t SC = f2_pack(sc, sc), NB = f2_pack(-base, -base);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t pw[16];
-#pragma unroll
-          for (int e2 = 0; e2 < 16; ++e2) {
-            float x0, x1;
-            f2_unpack(f2_fma(f2_pack(__uint_as_float(v[c][2 * e2]), __uint_as_float(v[c][2 * e2 + 1])), SC, NB),
-                      x0, x1);
-            const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-            L[e2 & 3] = f2_add(L[e2 & 3], f2_pack(p0, p1));
-            pw[e2] = pack_x2<F16>(p0, p1);
-          }
-          if (c == 2) {
-            // keys 0..63 are stored: hand them to the MMA before the rest
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(kBarP + 2 * i));
-          }
-          tmem_st16(tS + 16 * c, pw);
-        }
-        float l0, l1, l2, l3;
-        f2_unpack(f2_add(L[0], L[1]), l0, l1);
-        f2_unpack(f2_add(L[2], L[3]), l2, l3);
-        l_sum += (l0 + l1) + (l2 + l3);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(kBarP + 2 * i + 1));  // one arrival per warp, 4 per tile
-      }
-      if (!ok) *s_abort = 1;
-      // ---- epilogue: O / l --------------------------------------------------------
-      if (mbar_wait(bar(kBarO + i), 0, a.status) && ok && !*s_abort) {
-        tc_fence_after();
-        const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
-        const int64_t orow_i = q_row0 + (int64_t)i * a.N + r;
-        uint16_t* orow = a.out + orow_i * kHeadDim;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + 32 * c, o);
+          for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, v[c]);
           tmem_wait_ld();
-          reg_fence32(o);
 #pragma unroll
-          for (int q8 = 0; q8 < 4; ++q8) {
-            uint4 w;
-            w.x = pack_x2<F16>(__uint_as_float(o[8 * q8 + 0]) * inv_l, __uint_as_float(o[8 * q8 + 1]) * inv_l);
-            w.y = pack_x2<F16>(__uint_as_float(o[8 * q8 + 2]) * inv_l, __uint_as_float(o[8 * q8 + 3]) * inv_l);
-            w.z = pack_x2<F16>(__uint_as_float(o[8 * q8 + 4]) * inv_l, __uint_as_float(o[8 * q8 + 5]) * inv_l);
-            w.w = pack_x2<F16>(__uint_as_float(o[8 * q8 + 6]) * inv_l, __uint_as_float(o[8 * q8 + 7]) * inv_l);
-            *reinterpret_cast<uint4*>(orow + 32 * c + 8 * q8) = w;
+          for (int c = 0; c < 4; ++c) reg_fence32(v[c]);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            if (mk[c] != 0xffffffffu) {
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                if (!((mk[c] >> e) & 1u)) v[c][e] = __float_as_uint(-INFINITY);
+            }
           }
+          // ---- row maximum of the raw scores
+          float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int e2 = 0; e2 < 16; ++e2)
+              mp[e2 & 3] = fmax3(mp[e2 & 3], __uint_as_float(v[c][2 * e2]), __uint_as_float(v[c][2 * e2 + 1]));
+          const float mr = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
+          const float mloc = mr == -INFINITY ? -INFINITY : mr * sc;
+          float alpha = 1.f;
+          bool rescale = false;
+          if (m_used == -INFINITY) {
+            m_used = mloc;  // first visible key of the row: O and l are still zero
+          } else if (mloc > m_used + kRescaleLog2) {
+            alpha = fast_exp2(m_used - mloc);
+            m_used = mloc;
+            rescale = true;
+          }
+          if (__any_sync(0xffffffffu, rescale)) {
+            // the previous PV of this tile completed before S of this block was committed
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+              uint32_t o[32];
+              tmem_ld32(tO + 32 * c, o);
+              tmem_wait_ld();
+              reg_fence32(o);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              tmem_st32(tO + 32 * c, o);
+            }
+          }
+          l_sum *= alpha;
+          const float base = (m_used == -INFINITY) ? 0.f : m_used;
+          // ---- p = exp2(s*sc - base), two scores per packed f32x2 FMA; P goes
+          // back as bf16 pairs into columns 0..63 of the row's S (all read).
+          uint64_t L[4] = {0ull, 0ull, 0ull, 0ull};
+          const uint64_t SC = f2_pack(sc, sc), NB = f2_pack(-base, -base);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t pw[16];
+#pragma unroll
+            for (int e2 = 0; e2 < 16; ++e2) {
+              float x0, x1;
+              f2_unpack(f2_fma(f2_pack(__uint_as_float(v[c][2 * e2]), __uint_as_float(v[c][2 * e2 + 1])), SC, NB),
+                        x0, x1);
+              const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+              L[e2 & 3] = f2_add(L[e2 & 3], f2_pack(p0, p1));
+              pw[e2] = pack_x2<F16>(p0, p1);
+            }
+            if (c == 2) {
+              // keys 0..63 are stored: hand them to the MMA before the rest
+              tmem_wait_st();
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(bar(kBarP + 2 * i));
+            }
+            tmem_st16(tS + 16 * c, pw);
+          }
+          float l0, l1, l2, l3;
+          f2_unpack(f2_add(L[0], L[1]), l0, l1);
+          f2_unpack(f2_add(L[2], L[3]), l2, l3);
+          l_sum += (l0 + l1) + (l2 + l3);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(kBarP + 2 * i + 1));  // one arrival per warp, 4 per tile
         }
-        if (a.lse) a.lse[orow_i] = l_sum > 0.f ? (m_used + __log2f(l_sum)) * kLn2 : -INFINITY;
+        ok = __all_sync(0xffffffffu, ok && !*s_abort);
+        if (!ok) *s_abort = 1;
+        // ---- epilogue: O / l ------------------------------------------------------
+        // Each warp stages its 32 rows, 64 columns at a time, in the 128-byte-
+        // swizzled box layout and writes them with a TMA store (whole lines,
+        // asynchronous); before refilling its buffer it waits until the previous
+        // store has read it.  Only warp-level synchronisation is involved.
+        const bool ep = __all_sync(0xffffffffu, mbar_wait(bar(kBarO + i), pos & 1, a.status) && ok && !*s_abort);
+        if (ep) {
+          tc_fence_after();
+          const AttnItem it = attn_item_of<GATHER>(a, item, ntile, kt, am);
+          const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
+          const uint32_t stg = sbase + kAttnStage + (uint32_t)warp * kStageWarpBytes;  // warps 0-7
+          const int y = (int)(it.q_row0 + (int64_t)i * a.N) + 32 * (warp & 3);
+#pragma unroll 1
+          for (int hh = 0; hh < 2; ++hh) {
+            if (lane == 0) bulk_wait_read0();
+            __syncwarp();
+#pragma unroll
+            for (int c2 = 0; c2 < 2; ++c2) {
+              uint32_t o[32];
+              tmem_ld32(tO + 32 * (2 * hh + c2), o);
+              tmem_wait_ld();
+              reg_fence32(o);
+#pragma unroll
+              for (int q8 = 0; q8 < 4; ++q8) {
+                uint4 w;
+                w.x = pack_x2<F16>(__uint_as_float(o[8 * q8 + 0]) * inv_l, __uint_as_float(o[8 * q8 + 1]) * inv_l);
+                w.y = pack_x2<F16>(__uint_as_float(o[8 * q8 + 2]) * inv_l, __uint_as_float(o[8 * q8 + 3]) * inv_l);
+                w.z = pack_x2<F16>(__uint_as_float(o[8 * q8 + 4]) * inv_l, __uint_as_float(o[8 * q8 + 5]) * inv_l);
+                w.w = pack_x2<F16>(__uint_as_float(o[8 * q8 + 6]) * inv_l, __uint_as_float(o[8 * q8 + 7]) * inv_l);
+                const uint32_t chunk = (uint32_t)(4 * c2 + q8) ^ (uint32_t)(lane & 7);
+                sts128(stg + (uint32_t)lane * 128u + (chunk << 4), w);
+              }
+            }
+            fence_proxy_async_smem();  // the TMA store reads the staged rows through the async proxy
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tm_o, stg, 64 * hh, y);
+              bulk_commit();
+            }
+          }
+          if (a.lse) a.lse[it.q_row0 + (int64_t)i * a.N + r] = l_sum > 0.f ? (m_used + __log2f(l_sum)) * kLn2 : -INFINITY;
+        } else {
+          ok = false;
+        }
+        if (!__all_sync(0xffffffffu, ok)) break;
+        g += (uint32_t)nblk;
+        int nx = -1;
+        if (lane == 0) nx = read_item(pos, kt, am);
+        nx = __shfl_sync(0xffffffffu, nx, 0);
+        kt = __shfl_sync(0xffffffffu, kt, 0);
+        am = __shfl_sync(0xffffffffu, am, 0);
+        if (nx < 0) break;
+        item = nx;
       }
+      if (lane == 0) bulk_wait0();  // this warp's O stores have completed
     }
   }
   tc_fence_before();
@@ -873,9 +1098,10 @@ static cudaError_t launch_attn(const PrefillParams& p, bool gather, cudaStream_t
   const int n_tiles = p.N / kTile;
   const uint64_t kv_rows = (uint64_t)p.B * p.Hkv * p.N;
   if (kv_rows >= (1ull << 31) || (uint64_t)p.B * p.Hq * p.N >= (1ull << 31)) return cudaErrorNotSupported;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (!make_tile_map(&tq, p.q, (uint64_t)p.B * p.Hq * p.N, 128, p.f16) ||
-      !make_tile_map(&tk, p.k, kv_rows, 128, p.f16) || !make_tile_map(&tv, p.v, kv_rows, 128, p.f16))
+      !make_tile_map(&tk, p.k, kv_rows, 128, p.f16) || !make_tile_map(&tv, p.v, kv_rows, 128, p.f16) ||
+      !make_tile_map(&to, p.out, (uint64_t)p.B * p.Hq * p.N, 32, p.f16))
     return cudaErrorInvalidValue;
   AttnArgs a;
   a.B = p.B; a.Hq = p.Hq; a.Hkv = p.Hkv; a.G = p.G; a.N = p.N; a.n_tiles = n_tiles;
@@ -898,7 +1124,7 @@ static cudaError_t launch_attn(const PrefillParams& p, bool gather, cudaStream_t
   if (fa.numRegs != kLaunchRegs) return cudaErrorNotSupported;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kAttnThreads, kAttnSmem, st>>>(tq, tk, tv, a);
+  kern<<<grid, kAttnThreads, kAttnSmem, st>>>(tq, tk, tv, to, a);
   return cudaGetLastError();
 }
 
