@@ -139,6 +139,7 @@ struct AttnArgs {
   const int32_t* idx_k;
   const int32_t* head_map;
   int k_max;
+  int head_major;  // anchor item order: key head by key head (set when K/V exceed half of L2)
   float scale_log2;
   uint16_t* out;
   float* lse;
@@ -178,6 +179,10 @@ __device__ __forceinline__ constexpr uint64_t qpair_step(int ks) {
 // Item order (the grid's, kept by taking over pending CTAs in launch order):
 // anchor: longest tiles first over the whole grid (every head group and
 // sequence of tile t before any of tile t - 1), so no long tile starts late;
+// when all heads' K/V exceed half of L2, key head by key head instead
+// (longest tiles first within each), so the K/V being re-read by the running
+// CTAs stays in L2 (131K tokens: 204.4 against 211.9 ms; at 16K the global
+// order is 1-2% faster);
 // reuse: tiles longest first within each head group, the head groups one
 // after another (the CTAs running together then gather from the same key
 // head's rows, which measured faster than the global order).
@@ -202,6 +207,12 @@ __device__ __forceinline__ AttnItem attn_item_of(const AttnArgs& a, int item, in
   if (GATHER) {
     w.t = a.n_tiles - 1 - item % a.n_tiles;
     rem = item / a.n_tiles;
+  } else if (a.head_major) {
+    const int PH = HG / a.Hkv;  // head pairs per key head
+    const int p = item % PH, rest = item / PH;
+    w.t = a.n_tiles - 1 - rest % a.n_tiles;
+    const int bh = rest / a.n_tiles;
+    rem = (bh / a.Hkv) * HG + (bh % a.Hkv) * PH + p;
   } else {
     w.t = a.n_tiles - 1 - item / (HG * a.B);
     rem = item % (HG * a.B);
@@ -1107,6 +1118,7 @@ static cudaError_t launch_attn(const PrefillParams& p, bool gather, cudaStream_t
   a.B = p.B; a.Hq = p.Hq; a.Hkv = p.Hkv; a.G = p.G; a.N = p.N; a.n_tiles = n_tiles;
   a.k = p.k; a.v = p.v;
   a.idx = p.idx; a.idx_k = p.idx_k; a.head_map = p.head_map; a.k_max = p.k_max;
+  a.head_major = !gather && kv_rows * (uint64_t)kHeadDim * 2u * 2u > (64ull << 20);
   a.scale_log2 = (float)((double)p.scale * 1.4426950408889634);
   a.out = p.out; a.lse = p.lse; a.status = p.status;
   const int ntile = p.G >= 2 ? 2 : 1;
