@@ -221,3 +221,47 @@ def test_prefill_reuse_bad_index_sets_status():
     hm = torch.arange(cfg.Hkv, dtype=torch.int32)
     api.prefill_reuse(inp["q"], inp["k"], inp["v"], idx.to(DEV), idx_k.to(DEV), hm.to(DEV), SCALE)
     assert api.device_status() == 5
+
+
+def test_prefill_reuse_bad_rows_with_taken_over_items():
+    """Bad index data in a grid large enough that CTAs take over other CTAs'
+    items (N = 4096: 512 items).  Reuse key head 3 maps to an anchor head out
+    of range, and one index count exceeds its tile's prefix.  The call must
+    end with the bad-index status, not a timeout; the items those rows feed
+    fall back to the diagonal block alone (finite output); every other item
+    is bit-identical to a clean run."""
+    cfg = workload.scaled(workload.PREFILL_16K, name="prefill_bad_many", N=4096)
+    nt, G = cfg.N // TILE, cfg.Hq // cfg.Hkv
+    sch = PrefillSchedule(1, cfg.Hq, cfg.Hkv, cfg.N, (0,), 2, DEV)
+    a_in = workload.prefill_layer(cfg, 0, DEV)
+    sch.run_anchor(a_in, torch.empty_like(a_in["q"]))
+    sch.run_topk()
+    r_in = workload.prefill_layer(cfg, 1, DEV)
+    hm = workload.head_map(cfg, 1).to(DEV)
+    clean, lse_clean = api.prefill_reuse(r_in["q"], r_in["k"], r_in["v"], sch.idx, sch.row_k, hm, SCALE)
+    assert api.device_status() == 0
+
+    hm_bad = hm.clone()
+    hm_bad[3] = cfg.Hkv + 1
+    t_bad, h_bad = 20, 5
+    am = int(hm[h_bad])
+    rk_bad = sch.row_k.clone().view(1, nt, cfg.Hkv)
+    rk_bad[0, t_bad, am] = TILE * t_bad + 1
+    out, lse = api.prefill_reuse(r_in["q"], r_in["k"], r_in["v"], sch.idx, rk_bad.view(-1), hm_bad, SCALE)
+    assert api.device_status() == 5  # bad index, and no wait gave up
+
+    assert torch.isfinite(out.float()).all()
+    hm_np = hm.cpu().numpy()
+    for h in range(cfg.Hkv):
+        heads = slice(G * h, G * h + G)
+        if h == 3:
+            continue
+        if hm_np[h] == am:  # fed by the bad row at tile t_bad only
+            keep = torch.ones(cfg.N, dtype=torch.bool)
+            keep[TILE * t_bad:TILE * (t_bad + 1)] = False
+            keep = keep.to(DEV)
+            assert torch.equal(out[0, heads][:, keep], clean[0, heads][:, keep])
+            assert torch.equal(lse[0, heads][:, keep], lse_clean[0, heads][:, keep])
+        else:
+            assert torch.equal(out[0, heads], clean[0, heads])
+            assert torch.equal(lse[0, heads], lse_clean[0, heads])
