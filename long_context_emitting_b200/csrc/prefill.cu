@@ -374,6 +374,7 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       prefetch_rows(it, 1);
       uint32_t g = 0;            // key blocks of the CTA's earlier items
       int unread = -1;           // leader: a request whose response it has not read
+      bool q_pending = false;    // leader: this item's query tiles still to load
       if (leader) load_q(it);  // later items' tiles are loaded as the previous item ends
       for (int pos = 0;; ++pos) {
         bool ok = !__any_sync(0xffffffffu, *s_abort != 0);
@@ -434,6 +435,11 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
               tma_load_2d(vb, &tm_v, 0, y, bar(kBarKvFull + st));
               tma_load_2d(vb + kHalfBytes, &tm_v, 64, y, bar(kBarKvFull + st));
             }
+            if (leader && q_pending) {
+              if (mbar_wait(bar(kBarQFree), (pos - 1) & 1, a.status)) load_q(it);
+              else *s_abort = 1;
+              q_pending = false;
+            }
           } else {
             // Copy: each warp instruction moves two whole 256-byte rows (16 lanes per
             // row, one 16-byte chunk each) into the swizzled layout; masked rows are
@@ -467,6 +473,11 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 for (int e = 0; e < 4; ++e) masks[st * 4 + e] = m[e];
               }
               mbar_arrive(bar(kBarKvFull + st));  // release: rows (and masks) visible
+            }
+            if (leader && q_pending) {
+              if (mbar_wait(bar(kBarQFree), (pos - 1) & 1, a.status)) load_q(it);
+              else *s_abort = 1;
+              q_pending = false;
             }
           }
         }
@@ -503,15 +514,15 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         if (nx < 0 || __any_sync(0xffffffffu, *s_abort != 0)) break;
         it = attn_item_of<GATHER>(a, nx, ntile, nkt, nam);
         if (leader) {
-          // its query tiles: toward L2 at once, into shared memory as soon as
-          // this item's last S MMAs have completed
+          // its query tiles: toward L2 at once; into shared memory once its first
+          // K/V block is on its way and this item's last S MMAs have completed
+          // (both are needed by the item's first S MMA, so their loads overlap)
           for (int i = 0; i < ntile; ++i) {
             const int y = (int)(it.q_row0 + (int64_t)i * a.N);
             tma_prefetch_l2_2d(&tm_q, 0, y);
             tma_prefetch_l2_2d(&tm_q, 64, y);
           }
-          if (mbar_wait(bar(kBarQFree), pos & 1, a.status)) load_q(it);
-          else *s_abort = 1;
+          q_pending = true;  // loaded once this item's first K/V block is on its way
         }
         if (__any_sync(0xffffffffu, *s_abort != 0)) break;
         prefetch_rows(it, 0);
