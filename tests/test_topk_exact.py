@@ -94,3 +94,19 @@ def test_topk_bad_k_sets_status_and_fills_minus_one():
     assert api.device_status() == 5
     assert (got[0] == -1).all()
     assert got[1, :3].tolist() == O.topk_select(s[1].numpy(), 3).tolist()
+
+
+@pytest.mark.parametrize("sign", [1.0, -1.0], ids=["pos", "neg"])
+def test_topk_rows_with_long_common_prefixes(sign):
+    """Rows whose keys differ only in their last `bits` bits (1 .. 23): the radix
+    digits start below the shared prefix, with widths from 1 to 11 bits."""
+    rng = np.random.default_rng(20251218)
+    rows = []
+    for bits in (1, 2, 3, 10, 11, 12, 21, 22, 23):
+        base = np.array([sign * 0.37], dtype=np.float32).view(np.uint32)[0]
+        hi = base & np.uint32(~((1 << bits) - 1) & 0xFFFFFFFF)
+        low = rng.integers(0, 1 << bits, size=4096, dtype=np.uint64).astype(np.uint32)
+        rows.append((hi | low).view(np.float32))
+    scores = torch.from_numpy(np.stack(rows))
+    n = len(rows)
+    _check(scores, [4096] * n, [410, 1, 4095, 2048, 128, 3000, 7, 410, 4000][:n])
