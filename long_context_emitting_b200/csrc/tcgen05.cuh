@@ -1,5 +1,6 @@
 // Thin wrappers over the sm_100a PTX used by the prefill kernels: mbarriers,
-// TMA tile loads (no multicast), cp.async, and the tcgen05 tensor-core /
+// TMA tile loads (no multicast), stores and L2 prefetches, cp.async, cluster
+// launch control (taking over pending CTAs), and the tcgen05 tensor-core /
 // tensor-memory instructions.  Every wait is bounded (see mbar_wait).
 #pragma once
 
