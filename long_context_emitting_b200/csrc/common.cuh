@@ -15,6 +15,30 @@ constexpr unsigned kStatusBadIndex = 1u;
 constexpr unsigned kStatusNonFinite = 2u;
 constexpr unsigned kStatusTimeout = 4u;  // a bounded wait gave up
 
+// Programmatic dependent launch.  The decode reuse (gather) kernel is launched
+// with the programmatic stream-serialization attribute, so its CTAs can be
+// scheduled while the previous kernel of the stream (often the previous
+// layer's gather) finishes.  grid_dependency_wait() blocks until that kernel
+// has completed and its writes are visible (a no-op without the attribute);
+// the kernel calls it before its first global-memory access, so the stream's
+// order of effects is unchanged.  allow_dependents_launch() lets the next such
+// kernel start launching once every CTA of this grid has called it or exited.
+// (Giving the attribute to the decode anchor's split and combine kernels and
+// to Top-k as well made the 32-layer step 20% slower, so only the gather
+// kernel takes it.)
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// The launch attribute of programmatic dependent launch.
+inline cudaLaunchAttribute pdl_attribute() {
+  cudaLaunchAttribute at;
+  at.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at.val.programmaticStreamSerializationAllowed = 1;
+  return at;
+}
+
 __device__ __forceinline__ void flag_status(unsigned* status, unsigned bit) {
   if (status) atomicOr(status, bit);
 }

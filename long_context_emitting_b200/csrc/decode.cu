@@ -348,6 +348,7 @@ __device__ __forceinline__ uint32_t gswz(int r, int c) {
 
 template <bool PAGED, bool F16>
 __global__ void __launch_bounds__(kThreads, 3) decode_gather_kernel(const SplitArgs a) {
+  grid_dependency_wait();
   extern __shared__ uint8_t gsm_raw[];
   uint8_t* gsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gsm_raw) + 127) & ~uintptr_t(127));
   __shared__ uint32_t smask[kWarps][kGStages];
@@ -462,6 +463,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_gather_kernel(const SplitA
     compute_blk<true, F16>(x, ws, qf, a.scale_log2, nullptr, G, tig);
   }
   cp_async_wait<0>();
+  allow_dependents_launch();
 
   // ---- merge the 4 warps (the rings are free now) ---------------------------
   const float lsum0 = warp_sum_xor_gid(ws.l0);
@@ -746,13 +748,14 @@ static cudaError_t launch_decode(const DecodeParams& p, bool gather, cudaStream_
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = kGSmem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = sp.nsplit;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1] = pdl_attribute();
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     e = cudaLaunchKernelEx(&cfg, kern, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
