@@ -132,6 +132,14 @@ def test_prefill_n16384_sampled_tiles():
     _check(workload.PREFILL_16K, tiles=[0, 1, 10, 11, 64, 127])
 
 
+def test_prefill_b2_n16384_key_head_order_sampled_tiles():
+    # two sequences of 16K: all heads' K/V exceed half of L2, so the anchor
+    # attention takes its items key head by key head; tiles of the second
+    # sequence check that order's (sequence, head) mapping
+    cfg = workload.scaled(workload.PREFILL_16K, name="prefill_b2_n16384", B=2)
+    _check(cfg, tiles=[0, 5, 64, 127], b=1)
+
+
 def test_prefill_n65536_sampled_tiles():
     _check(workload.PREFILL_64K, tiles=[0, 2, 300, 511])
 
