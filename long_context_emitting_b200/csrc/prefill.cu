@@ -361,7 +361,15 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       };
       // The item's query tiles (leader).  Their buffer is free once the previous
       // item's S MMAs have read it.
+      // leader: the loads an abort must wait for, two bits per barrier (issued,
+      // phase parity): field 0 the query tiles (kBarQ), 1 + s K/V stage s
+      uint32_t inflight = 0u;
+      auto note_load = [&](int field, uint32_t parity) {
+        inflight = (inflight & ~(3u << (2 * field))) | ((1u | (parity << 1)) << (2 * field));
+      };
       auto load_q = [&](const AttnItem& w) {
+        const uint32_t qf = inflight & 3u;
+        note_load(0, (qf & 1u) ? ((qf >> 1) ^ 1u) : 0u);  // the next kBarQ phase
         mbar_expect_tx(bar(kBarQ), ntile * kTileBytes);
         for (int i = 0; i < ntile; ++i) {
           const int y = (int)(w.q_row0 + (int64_t)i * a.N);
@@ -429,6 +437,7 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
               if (lane == 0) mbar_arrive(bar(kBarKvFull + st));  // helpers complete the count
             } else if (lane == 0) {
               mbar_expect_tx(bar(kBarKvFull + st), 2 * kTileBytes);
+              note_load(1 + st, (gb >> 1) & 1u);
               const int y = it.kv_row0 + kTile * (GATHER ? it.t : j);
               tma_load_2d(kb, &tm_k, 0, y, bar(kBarKvFull + st));
               tma_load_2d(kb + kHalfBytes, &tm_k, 64, y, bar(kBarKvFull + st));
@@ -530,6 +539,14 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       }
       // never leave with a response still to land in shared memory
       if (leader && unread >= 0) mbar_wait(bar(kBarClcFull + (unread & 1)), (unread >> 1) & 1, a.status);
+      // after an abort, wait (bounded) for the copies this thread started: the
+      // last query-tile load and the last TMA load into each stage (a gathered
+      // block's cp.async copies are waited for by the warps that issue them)
+      if (leader && *s_abort) {
+        for (int f = 0; f < 3; ++f)
+          if ((inflight >> (2 * f)) & 1u)
+            mbar_wait(bar(f == 0 ? kBarQ : kBarKvFull + f - 1), (inflight >> (2 * f + 1)) & 1u, a.status);
+      }
     } else if (warp == kMmaWarp) {
       // ================================ MMA issuer ==================================
       if (lane == 0) {
@@ -895,6 +912,8 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   // so the MMA fills one buffer while the summing warps work on the other.
   if (warp < 4) {
     setmaxnreg_dec<kPoolCtlRegs>();
+    int q_loads = 0;             // warp 0 lane 0: query-tile loads issued (one kPBarQ phase each)
+    int last_k0 = -1, last_k1 = -1;  // warp 0 lane 0: K-block counter of the last load into stage 0 / 1
     for (int rd = 0; rd < n_rounds; ++rd) {
       const int gbase = h * G + rd * kPoolHeads;
       const int kit0 = rd * nblk;  // running K-block counter (stage / phase bookkeeping)
@@ -902,6 +921,7 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       if (warp == 0) {
         // ---------------------------- TMA producer ----------------------------
         if (lane == 0) {
+          ++q_loads;
           mbar_expect_tx(bar(kPBarQ), hg * kTileBytes);
           for (int j = 0; j < hg; ++j) {
             const int y = (int)(((int64_t)b * a.Hq + gbase + j) * a.N + (int64_t)kTile * t);
@@ -914,6 +934,7 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (*s_abort) break;
             const uint32_t ks = sbase + kPoolK + st * kTileBytes;
             mbar_expect_tx(bar(kPBarKFull + st), kTileBytes);
+            if (st) last_k1 = kit; else last_k0 = kit;
             tma_load_2d(ks, &tm_k, 0, kv_row0 + kTile * jb, bar(kPBarKFull + st));
             tma_load_2d(ks + kHalfBytes, &tm_k, 64, kv_row0 + kTile * jb, bar(kPBarKFull + st));
           }
@@ -952,6 +973,13 @@ prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
       }
       __syncthreads();  // round done: Q tiles and the -lse tiles may be replaced
+    }
+    // after an abort, wait (bounded) for the copies the producer started: the
+    // last query-tile load and the last K load into each stage
+    if (warp == 0 && lane == 0 && *s_abort) {
+      if (q_loads > 0) mbar_wait(bar(kPBarQ), (uint32_t)(q_loads - 1) & 1u, a.status);
+      if (last_k0 >= 0) mbar_wait(bar(kPBarKFull + 0), ((uint32_t)last_k0 >> 1) & 1u, a.status);
+      if (last_k1 >= 0) mbar_wait(bar(kPBarKFull + 1), ((uint32_t)last_k1 >> 1) & 1u, a.status);
     }
   } else {
     setmaxnreg_inc<kPoolSumRegs>();
