@@ -79,9 +79,13 @@ class Dist:
         if self.world > 1:
             import datetime
             import torch.distributed as dist
-            torch.cuda.set_device(self.local)
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
-                                    device_id=torch.device("cuda", self.local))
+            if torch.cuda.is_available():
+                torch.cuda.set_device(self.local)
+                dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                        device_id=torch.device("cuda", self.local))
+            else:
+                # no GPU: only the reference arm (host cores) can run; gloo for its ranks
+                dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=600))
             self.pg = dist
 
     def barrier(self):
