@@ -199,7 +199,12 @@ int kascade_prefill_anchor(kascade_shape s, int32_t N, const uint16_t* q, const 
  *   q, k, v as in kascade_prefill_anchor
  *   idx int32 [B, N/128, Hkv, k_max]; idx_k int32 [B·(N/128)·Hkv]; head_map int32 [Hkv]
  *   out bf16 [B, Hq, N, d]; lse fp32 [B, Hq, N] (may be NULL)
- *   ws scratch of kascade_prefill_reuse_workspace_bytes(s, N, k_max) bytes */
+ *   ws scratch of kascade_prefill_reuse_workspace_bytes(s, N, k_max) bytes
+ *
+ * Device-side errors (KASCADE_ERR_BAD_INDEX in the status word): an index
+ * outside [0, 128t) is skipped; a head_map entry outside [0, Hkv), or an idx_k
+ * entry outside [0, min(k_max, 128t)], drops that row's whole index set, and
+ * its queries attend to their diagonal block alone. */
 size_t kascade_prefill_reuse_workspace_bytes(kascade_shape s, int32_t N, int32_t k_max);
 int kascade_prefill_reuse(kascade_shape s, int32_t N, const uint16_t* q, const uint16_t* k,
                           const uint16_t* v, const int32_t* idx, const int32_t* idx_k,
