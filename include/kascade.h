@@ -100,7 +100,7 @@ int kascade_decode_anchor(kascade_shape s, const uint16_t* q, const uint16_t* k,
 /* Size of the library-owned scratch array used by kascade_decode_anchor_static_ws. */
 #define KASCADE_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
 
-/* Decode anchor without caller-provided scratch.  The paper has no counterpart of
+/* Decode anchor without caller-provided scratch.  The method has no counterpart of
  * this entry point; it exists for callers that cannot allocate device memory at
  * the point where they run the layer: an inference-runtime plugin whose enqueue
  * step may not allocate, or a serving engine that has handed nearly all device
